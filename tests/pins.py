@@ -1,0 +1,330 @@
+"""Pins of the CPU oracle: checks against things other than the oracle itself.
+
+Each `pin_*` takes a compiled oracle (the real one, or a planted-mistake
+mutant) and returns True when the oracle agrees with what the binary16 format,
+the packing rule, exact arithmetic or a library routine fixes. The pytest
+wrappers in test_oracle_pins.py assert each one on the real oracle; the mutant
+test asserts that every planted mistake makes at least one of them fail.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+
+import workloads
+from oracle import exact
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _read_table(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+def python_pack(q: np.ndarray) -> np.ndarray:
+    """The canonical packing rule, written independently for cross-checks."""
+    K, N = q.shape
+    out = np.zeros(((K + 1) // 2, N), dtype=np.uint8)
+    u = q.astype(np.int16) & 0xF
+    out[:] = u[0::2]
+    if K > 1:
+        out[: K // 2] |= (u[1::2] << 4).astype(np.uint8)
+    return out
+
+
+def decode_tiled(wt: np.ndarray, K: int, N: int) -> np.ndarray:
+    """Read every code back out of the tiled layout by its position formula."""
+    KT = (K + 63) // 64
+    perm = (0, 2, 4, 6, 1, 3, 5, 7)
+    pos = {r: i for i, r in enumerate(perm)}
+    q = np.zeros((K, N), dtype=np.int8)
+    for k in range(K):
+        kt, kl = divmod(k, 64)
+        h, r32 = divmod(kl, 32)
+        w, r = divmod(r32, 8)
+        i = pos[r]
+        for n in range(N):
+            nt, j = divmod(n, 128)
+            b = int(wt[(nt * KT + kt) * 4096 + h * 2048 + j * 16 + w * 4 + i // 2])
+            v = (b >> 4) if (i & 1) else (b & 0xF)
+            q[k, n] = v - 16 if v >= 8 else v
+    return q
+
+
+# ---------------------------------------------------------------- binary16
+
+def pin_half_widening(o) -> bool:
+    """All 65536 binary16 patterns widen exactly as numpy's float16 -> float64 does."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    for b in range(0, 65536, 1):
+        got = o.half_to_double(b)
+        r = ref[b]
+        if np.isnan(r):
+            if not np.isnan(got):
+                return False
+        elif got != r or np.signbit(got) != np.signbit(r):
+            return False
+    return True
+
+
+def _rounding_probe_values(seed=7):
+    """Doubles at, just above and just below binary16 rounding ties, plus random ones."""
+    g = np.random.Generator(np.random.PCG64(seed))
+    h = g.integers(0, 0x7BFF, size=3000).astype(np.uint16)  # finite positive patterns
+    lo = h.view(np.float16).astype(np.float64)
+    hi = (h + 1).view(np.float16).astype(np.float64)
+    mid = (lo + hi) / 2.0  # exact in double
+    vals = [mid, np.nextafter(mid, np.inf), np.nextafter(mid, -np.inf), lo, -mid,
+            g.standard_normal(2000) * 10.0 ** g.integers(-9, 5, size=2000)]
+    return np.concatenate(vals)
+
+
+def pin_half_rounding(o) -> bool:
+    """double -> binary16 agrees with exact integer RNE on ties and near-ties."""
+    for x in _rounding_probe_values():
+        x = float(x)
+        if not np.isfinite(x) or x == 0.0:
+            continue
+        m, e = np.frexp(x)
+        # x = mant * 2^(e-53) exactly, mant an integer
+        mant = int(np.ldexp(m, 53))
+        want = exact.round_units_to_half(mant, int(e) - 53)
+        if o.double_to_half(x) != want:
+            return False
+    return True
+
+
+def pin_half_rounding_numpy(o) -> bool:
+    """double -> binary16 agrees with numpy's direct float64 -> float16 cast."""
+    vals = _rounding_probe_values(seed=8)
+    want = vals.astype(np.float16).view(np.uint16)
+    return all(o.double_to_half(float(x)) == int(w) for x, w in zip(vals, want))
+
+
+# ----------------------------------------------------------------- packing
+
+def pin_pack_golden(o) -> bool:
+    rows = _read_table("pack_bytes.txt")
+    q = np.array([[int(r[0]) for r in rows], [int(r[1]) for r in rows]], dtype=np.int8)
+    want = np.array([int(r[2], 16) for r in rows], dtype=np.uint8)
+    return bool(np.array_equal(o.pack(q)[0], want))
+
+
+def pin_pack_all_bytes(o) -> bool:
+    """Every byte value unpacks to two codes in [-8, 7] and packs back to itself."""
+    wp = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    q = o.unpack(wp, 2)
+    if q.min() < -8 or q.max() > 7:
+        return False
+    if not np.array_equal(o.pack(q), wp):
+        return False
+    # low nibble is the even row, as a two's-complement nibble
+    lo = np.arange(256) & 0xF
+    return bool(np.array_equal(q[0], np.where(lo >= 8, lo - 16, lo)))
+
+
+def pin_pack_random_odd_k(o) -> bool:
+    """Random codes with odd K: pack equals the independent rule, unpack inverts it."""
+    g = np.random.Generator(np.random.PCG64(5))
+    q = g.integers(-8, 8, size=(37, 29), dtype=np.int8)
+    wp = o.pack(q)
+    if not np.array_equal(wp, python_pack(q)):
+        return False
+    if np.any(wp[-1] >> 4):  # no odd row beyond K
+        return False
+    return bool(np.array_equal(o.unpack(wp, 37), q))
+
+
+def pin_tiled_positions(o) -> bool:
+    """A single code lands at the byte and nibble its position formula gives."""
+    K, N = 100, 200
+    for k, n, byte, half in _read_table("tiled_positions.txt"):
+        q = np.zeros((K, N), dtype=np.int8)
+        q[int(k), int(n)] = 5
+        wt = o.tile(q)
+        nz = np.nonzero(wt)[0]
+        want = 0x05 if half == "low" else 0x50
+        if len(nz) != 1 or nz[0] != int(byte) or wt[nz[0]] != want:
+            return False
+    return True
+
+
+def pin_tiled_roundtrip(o) -> bool:
+    """Random codes, ragged K and N: decoding the tiles by formula returns q."""
+    g = np.random.Generator(np.random.PCG64(6))
+    q = g.integers(-8, 8, size=(72, 136), dtype=np.int8)
+    wt = o.tile(q)
+    return len(wt) == o.tiled_bytes(72, 136) == 2 * 2 * 4096 and \
+        bool(np.array_equal(decode_tiled(wt, 72, 136), q))
+
+
+# ----------------------------------------------------------------- product
+
+def pin_exact_small(o) -> bool:
+    """Bit-exact against the integer brute force on small ragged shapes."""
+    for (M, K, N, G, seed) in [(3, 40, 9, 16, 1), (2, 65, 7, 13, 2), (4, 96, 16, 32, 3),
+                               (1, 7, 5, 3, 4)]:
+        c = workloads.dense(M, K, N, G, seed)
+        got = o.gemm(c.A, python_pack(c.q), c.S, K, G)
+        want = exact.gemm_exact(c.A, c.q, c.S, G)
+        if not np.array_equal(got.view(np.uint16), want.view(np.uint16)):
+            return False
+    return True
+
+
+def pin_exact_tiny_config(o, cols=None) -> bool:
+    """Bit-exact against the integer brute force on the tiny config (4x512x512, G=128)."""
+    c = workloads.make("tiny")
+    cols = slice(None) if cols is None else cols
+    q = c.q[:, cols]
+    S = c.S[:, cols]
+    got = o.gemm(c.A, python_pack(q), S, c.K, c.G)
+    want = exact.gemm_exact(c.A, q, S, c.G)
+    return bool(np.array_equal(got.view(np.uint16), want.view(np.uint16)))
+
+
+def pin_near_ties(o) -> bool:
+    with open(os.path.join(GOLDEN, "near_ties.json")) as f:
+        cases = json.load(f)["cases"]
+    for cs in cases:
+        K, G = cs["K"], cs["G"]
+        A = np.array([cs["A"]], dtype=np.float16).reshape(cs["M"], K)
+        q = np.array(cs["q"], dtype=np.int8)
+        S = np.array(cs["S"], dtype=np.float16)
+        got = o.gemm(A, python_pack(q), S, K, G).view(np.uint16)
+        want = np.array([[int(x, 16) for x in row] for row in cs["C_bits"]], dtype=np.uint16)
+        if not np.array_equal(got, want):
+            return False
+    return True
+
+
+def pin_closed_form(o) -> bool:
+    """Constant q and s: C[m, n] = fp16(q * s * sum_k A[m, k]) for every n."""
+    M, K, N, G = 3, 192, 6, 64
+    g = np.random.Generator(np.random.PCG64(9))
+    A = g.standard_normal((M, K), dtype=np.float32).astype(np.float16)
+    for qv, sv in [(-3, 0.0107421875), (7, 0.003), (-8, 0.019)]:
+        s16 = np.float16(sv)
+        q = np.full((K, N), qv, dtype=np.int8)
+        S = np.full((-(-K // G), N), s16, dtype=np.float16)
+        got = o.gemm(A, python_pack(q), S, K, G).view(np.uint16)
+        s_units = exact.half_to_units(int(np.array(s16).view(np.uint16)))
+        for m in range(M):
+            row_units = sum(exact.half_to_units(int(b)) for b in A[m].view(np.uint16))
+            want = exact.round_units_to_half(row_units * qv * s_units, -48)
+            if not np.all(got[m] == want):
+                return False
+    return True
+
+
+def pin_one_hot(o) -> bool:
+    """s = 1 and q[k, n] = 1 only at k = pi(n): C[m, n] = A[m, pi(n)] exactly."""
+    M, K, N, G = 5, 130, 12, 64
+    g = np.random.Generator(np.random.PCG64(10))
+    A = g.standard_normal((M, K), dtype=np.float32).astype(np.float16)
+    # even and odd rows, rows in the second byte of a group, the last row
+    pi = np.array([0, 1, 2, 3, 63, 64, 65, 127, 128, 129, 77, 30])
+    q = np.zeros((K, N), dtype=np.int8)
+    q[pi, np.arange(N)] = 1
+    S = np.ones((-(-K // G), N), dtype=np.float16)
+    got = o.gemm(A, python_pack(q), S, K, G)
+    return bool(np.array_equal(got.view(np.uint16), A[:, pi].view(np.uint16)))
+
+
+def pin_scale_duplication(o) -> bool:
+    """G = K with scale row s0 equals G = 64 and G = 128 with s0 repeated in every group."""
+    M, K, N = 3, 256, 10
+    c = workloads.dense(M, K, N, K, 11)
+    wp = python_pack(c.q)
+    base = o.gemm(c.A, wp, c.S, K, K)
+    for G in (64, 128):
+        S = np.repeat(c.S, K // G, axis=0)
+        if not np.array_equal(o.gemm(c.A, wp, S, K, G).view(np.uint16), base.view(np.uint16)):
+            return False
+    # and a single nonzero-scale group selects exactly that group's rows
+    G = 64
+    S = np.zeros((K // G, N), dtype=np.float16)
+    S[2] = c.S[0]
+    q2 = c.q.copy()
+    q2[:128] = 0
+    q2[192:] = 0
+    want = o.gemm(c.A, python_pack(q2), c.S, K, K)
+    return bool(np.array_equal(o.gemm(c.A, wp, S, K, G).view(np.uint16), want.view(np.uint16)))
+
+
+def dequant_numpy(q: np.ndarray, S: np.ndarray, G: int) -> np.ndarray:
+    """float64 dequantised weights from the int8 codes, without the oracle."""
+    rows = np.arange(q.shape[0]) // G
+    return q.astype(np.float64) * S.astype(np.float64)[rows]
+
+
+def pin_numpy_blas(o) -> bool:
+    """numpy float64 matmul of the dequantised weights, rounded to fp16, agrees to 1 ulp."""
+    c = workloads.dense(6, 320, 48, 64, 12)
+    got = o.gemm(c.A, python_pack(c.q), c.S, c.K, c.G).view(np.uint16).astype(np.int32)
+    ref = (c.A.astype(np.float64) @ dequant_numpy(c.q, c.S, c.G)).astype(np.float16)
+    want = ref.view(np.uint16).astype(np.int32)
+    # same sign, at most one step apart in the ordered binary16 encoding
+    return bool(np.all(np.abs(got - want) <= 1))
+
+
+def pin_grouped_segments(o) -> bool:
+    """Grouped form: each segment (an empty expert included) equals the plain product on its
+    rows, and E=1 with one segment over all rows is the plain product."""
+    c = workloads.grouped(E=4, top_k=2, tokens=9, K=64, N=24, G=32, seed=13, empty_experts=[2])
+    wps = [python_pack(c.q[e]) for e in range(c.E)]
+    sentinel = np.full((c.total_rows, c.N), np.float16(-7.5))
+    got = o.grouped_gemm(c.A, wps, list(c.S), c.offsets, c.K, c.G, C=sentinel)
+    if c.offsets[2] != c.offsets[3]:
+        return False
+    for e in range(c.E):
+        r0, r1 = c.offsets[e], c.offsets[e + 1]
+        if r1 > r0:
+            want = o.gemm(c.A[r0:r1], wps[e], c.S[e], c.K, c.G)
+            if not np.array_equal(got[r0:r1].view(np.uint16), want.view(np.uint16)):
+                return False
+    one = o.grouped_gemm(c.A, wps[:1], [c.S[0]], np.array([0, c.total_rows]), c.K, c.G)
+    plain = o.gemm(c.A, wps[0], c.S[0], c.K, c.G)
+    if not np.array_equal(one.view(np.uint16), plain.view(np.uint16)):
+        return False
+    return True
+
+
+def pin_grouped_brute(o) -> bool:
+    """Grouped form against the integer brute force on each expert's rows."""
+    c = workloads.grouped(E=3, top_k=1, tokens=7, K=48, N=10, G=16, seed=14)
+    wps = [python_pack(c.q[e]) for e in range(c.E)]
+    got = o.grouped_gemm(c.A, wps, list(c.S), c.offsets, c.K, c.G)
+    for e in range(c.E):
+        r0, r1 = c.offsets[e], c.offsets[e + 1]
+        if r1 > r0:
+            want = exact.gemm_exact(c.A[r0:r1], c.q[e], c.S[e], c.G)
+            if not np.array_equal(got[r0:r1].view(np.uint16), want.view(np.uint16)):
+                return False
+    return True
+
+
+def pin_sample_matches_full(o) -> bool:
+    """The one-by-one sampler returns the same elements as the full product."""
+    c = workloads.dense(5, 200, 33, 40, 15)
+    wp = python_pack(c.q)
+    full = o.gemm(c.A, wp, c.S, c.K, c.G)
+    rows = [0, 4, 2, 3, 1, 4]
+    cols = [0, 32, 17, 5, 31, 1]
+    got = o.gemm_sample(c.A, wp, c.S, c.K, c.G, rows, cols)
+    return bool(np.array_equal(got.view(np.uint16), full[rows, cols].view(np.uint16)))
+
+
+PINS = [pin_half_widening, pin_half_rounding, pin_half_rounding_numpy, pin_pack_golden,
+        pin_pack_all_bytes, pin_pack_random_odd_k, pin_tiled_positions, pin_tiled_roundtrip,
+        pin_exact_small, pin_near_ties, pin_closed_form, pin_one_hot, pin_scale_duplication,
+        pin_numpy_blas, pin_grouped_segments, pin_grouped_brute, pin_sample_matches_full]

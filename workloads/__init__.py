@@ -1,0 +1,127 @@
+"""Seeded synthetic inputs for the W4A16 group-wise GEMM and its grouped-expert form.
+
+This module is shared by the CPU oracle's tests and by the CUDA path's tests and
+benchmark. It only draws random numbers and arranges them; it holds none of the
+method's arithmetic (no packing, no dequantisation, no products).
+
+Tensor roles and shapes follow the Int4GroupwiseGemmPluginV2 page (class
+description: activations [b, seq, K] fp16, scales [ceil(K/G), N] fp16, output
+[b, seq, N] fp16; constructor: N = columns, K = rows of the weight matrix,
+groupSize = G). The int4 codes are signed values in [-8, 7].
+
+Distributions (one seeded numpy PCG64 generator per case):
+  A  ~ N(0, 1) drawn in float32, rounded to float16
+  q  ~ uniform integers in [-8, 7]
+  s  ~ uniform in [0.002, 0.02] drawn in float32, rounded to float16
+Grouped-expert case (Int4MoePlugin page, constructor: numExperts, topK,
+hiddenSize, moeInterSize, quantizationGroupSize): each token draws topK distinct
+experts uniformly; the (token, slot) pairs are stably sorted by expert, which
+gives the gathered activation rows and the [E+1] prefix offsets.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, List, Optional
+
+import numpy as np
+
+S_LOW, S_HIGH = 0.002, 0.02
+
+
+def _rng(seed: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def n_groups(K: int, G: int) -> int:
+    return -(-K // G)
+
+
+@dataclasses.dataclass
+class DenseCase:
+    name: str
+    M: int
+    K: int
+    N: int
+    G: int
+    seed: int
+    A: np.ndarray  # [M, K] float16
+    q: np.ndarray  # [K, N] int8 in [-8, 7]
+    S: np.ndarray  # [ceil(K/G), N] float16
+
+
+@dataclasses.dataclass
+class GroupedCase:
+    name: str
+    E: int
+    top_k: int
+    tokens: int
+    K: int
+    N: int
+    G: int
+    seed: int
+    A_tokens: np.ndarray      # [tokens, K] float16
+    experts: np.ndarray       # [tokens, top_k] int32, distinct per token
+    order: np.ndarray         # [tokens*top_k] int64: flat (token*top_k + slot) index of each gathered row
+    A: np.ndarray             # [rows, K] float16, rows gathered per expert
+    offsets: np.ndarray       # [E+1] int32 prefix offsets into A's rows
+    q: np.ndarray             # [E, K, N] int8
+    S: np.ndarray             # [E, ceil(K/G), N] float16
+
+    @property
+    def total_rows(self) -> int:
+        return int(self.offsets[-1])
+
+
+def dense(M: int, K: int, N: int, G: int, seed: int, name: str = "dense",
+          a_scale: float = 1.0) -> DenseCase:
+    """One dense case with the distributions stated in the module docstring."""
+    g = _rng(seed)
+    A = (g.standard_normal((M, K), dtype=np.float32) * np.float32(a_scale)).astype(np.float16)
+    q = g.integers(-8, 8, size=(K, N), dtype=np.int8)
+    S = g.uniform(S_LOW, S_HIGH, size=(n_groups(K, G), N)).astype(np.float32).astype(np.float16)
+    return DenseCase(name, M, K, N, G, seed, A, q, S)
+
+
+def grouped(E: int, top_k: int, tokens: int, K: int, N: int, G: int, seed: int,
+            name: str = "grouped", empty_experts: Optional[List[int]] = None) -> GroupedCase:
+    """Top-k routing of `tokens` tokens over E experts, rows gathered per expert.
+
+    `empty_experts` (test aid) lists experts that no token may pick.
+    """
+    g = _rng(seed)
+    A_tokens = g.standard_normal((tokens, K), dtype=np.float32).astype(np.float16)
+    allowed = np.array([e for e in range(E) if not empty_experts or e not in empty_experts])
+    if top_k > len(allowed):
+        raise ValueError("top_k exceeds the number of selectable experts")
+    experts = np.stack([g.choice(allowed, size=top_k, replace=False) for _ in range(tokens)]).astype(np.int32)
+    flat = experts.reshape(-1)
+    order = np.argsort(flat, kind="stable")
+    counts = np.bincount(flat, minlength=E)
+    offsets = np.zeros(E + 1, dtype=np.int32)
+    offsets[1:] = np.cumsum(counts)
+    A = A_tokens[order // top_k]
+    q = g.integers(-8, 8, size=(E, K, N), dtype=np.int8)
+    S = g.uniform(S_LOW, S_HIGH, size=(E, n_groups(K, G), N)).astype(np.float32).astype(np.float16)
+    return GroupedCase(name, E, top_k, tokens, K, N, G, seed, A_tokens, experts,
+                       order.astype(np.int64), np.ascontiguousarray(A), offsets, q, S)
+
+
+# The five workload families and their sizes, with a fixed seed per config.
+CONFIGS: Dict[str, dict] = {
+    "tiny":        dict(kind="dense", M=4, K=512, N=512, G=128, seed=0),
+    "decode_m1":   dict(kind="dense", M=1, K=4096, N=4096, G=128, seed=1),
+    "decode_m16":  dict(kind="dense", M=16, K=4096, N=4096, G=128, seed=11),
+    "mlp_up":      dict(kind="dense", M=8, K=4096, N=14336, G=128, seed=2),
+    "mlp_down":    dict(kind="dense", M=8, K=14336, N=4096, G=128, seed=21),
+    "mlp_up_g64":  dict(kind="dense", M=8, K=4096, N=14336, G=64, seed=22),
+    "prefill":     dict(kind="dense", M=2048, K=4096, N=4096, G=128, seed=3),
+    "grouped":     dict(kind="grouped", E=8, top_k=2, tokens=512, K=4096, N=14336, G=128, seed=4),
+}
+
+
+def make(name: str):
+    cfg = dict(CONFIGS[name])
+    kind = cfg.pop("kind")
+    if kind == "dense":
+        return dense(name=name, **cfg)
+    return grouped(name=name, **cfg)
