@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A16 group-wise GEMM on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one step): the decode projection K = N = 4096, G = 128, run at M = 1
+and at M = 16 (two GEMM launches over the same weight shape). Inputs are seeded
+synthetic data with the distributions of the workloads module, resident in HBM
+before the timed region. Every launch reads a different one of R rotating
+copies of (tiled weights, scales, activations) whose total exceeds twice the
+L2 size, so no launch finds its weights in L2.
+
+The timed region replays CUDA graphs of the steps, bracketed by a barrier and
+torch.cuda.synchronize(); its time is the max over ranks (CUDA events). One
+JSON line goes to stdout on rank 0. `value` is effective HBM GB/s: algorithmic
+bytes (packed weights + scales + activations + output, each once) of all ranks'
+steps divided by that time. With --gpus N > 1 the ranks are independent
+replicas (the path has no exchange step).
+
+`--impl reference` times the CPU oracle (fp64, OpenMP) on a bounded column
+sample of the same step, on the host cores; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "W4A16 GEMM TFLOPS and effective HBM GB/s vs roofline, M=1..2048 (1 B200)"
+K_DIM, N_DIM, G_DIM = 4096, 4096, 128
+M_STEP = (1, 16)
+WORKLOAD = "decode projection: W4A16 GEMM at M=1 and at M=16, K=4096, N=4096, G=128 (one launch each per step)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GRAPH_CHUNK = 500
+
+
+def algorithmic_bytes(M, N, K, G):
+    """Packed int4 weights + fp16 scales + fp16 activations + fp16 output, each moved once."""
+    return (K * N) // 2 + (-(-K // G)) * N * 2 + M * K * 2 + M * N * 2
+
+
+def flops(M, N, K):
+    return 2 * M * N * K
+
+
+def step_bytes():
+    return sum(algorithmic_bytes(m, N_DIM, K_DIM, G_DIM) for m in M_STEP)
+
+
+def step_flops():
+    return sum(flops(m, N_DIM, K_DIM) for m in M_STEP)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples taken while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.25)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = list(csv.reader(io.StringIO(open(self.path).read())))
+        os.unlink(self.path)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ helpers
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def traffic_from_profile():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "weight_only_int4_wise_b200", "csrc", "w4a16_gemm.cu")
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if d.get("kernel_source_sha256") != digest:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def oracle_sample(o, case, cols):
+    """Packed weights and scales of the first `cols` columns (setup, outside any timing)."""
+    return o.pack(np.ascontiguousarray(case.q[:, :cols])), np.ascontiguousarray(case.S[:, :cols])
+
+
+def oracle_decode_step(o, case, sample):
+    """One decode step (M=1 and M=16) of the CPU oracle over a column sample."""
+    wp, S = sample
+    for m in M_STEP:
+        o.gemm(case.A[:m], wp, S, K_DIM, G_DIM)
+
+
+def sample_bytes(cols):
+    return sum(algorithmic_bytes(m, cols, K_DIM, G_DIM) for m in M_STEP)
+
+
+def cpu_baseline(budget_s=12.0):
+    import oracle
+    o = oracle.load()
+    case = workloads.dense(16, K_DIM, N_DIM, G_DIM, seed=1)
+    wp = o.pack(case.q)
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while True:
+        t0 = time.perf_counter()
+        for m in M_STEP:
+            o.gemm(case.A[:m], wp, case.S, K_DIM, G_DIM)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() > t_end or len(times) >= 20:
+            break
+    t = statistics.median(times)
+    return {"value": step_bytes() / t / 1e9, "unit": "GB/s", "cores": o.threads(), "kind": "oracle",
+            "sample": f"full decode step (M=1 and M=16, K=N=4096, G=128), median of {len(times)} runs, "
+                      f"{t * 1e3:.1f} ms per step"}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from weight_only_int4_wise_b200 import build as wbuild
+    wbuild.build()
+    import weight_only_int4_wise_b200 as w4
+
+    dev = torch.device("cuda", local)
+    case = workloads.dense(16, K_DIM, N_DIM, G_DIM, seed=1)
+    q = torch.from_numpy(case.q).to(dev)
+    _, wt0 = w4.prepare_weights(q)
+    S0 = torch.from_numpy(case.S).to(dev)
+    A0 = torch.from_numpy(case.A).to(dev)
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20)
+    copy_bytes = wt0.numel() + S0.numel() * 2 + A0.numel() * 2
+    R = max(3, math.ceil(2 * l2 / copy_bytes) + 1)
+    wts = [wt0] + [wt0.clone() for _ in range(R - 1)]
+    Ss = [S0] + [S0.clone() for _ in range(R - 1)]
+    As = [A0] + [A0.clone() for _ in range(R - 1)]
+    C1 = torch.empty((1, N_DIM), dtype=torch.float16, device=dev)
+    C16 = torch.empty((16, N_DIM), dtype=torch.float16, device=dev)
+    outs = {1: C1, 16: C16}
+
+    def launch(m, r):
+        rc = w4.w4a16_gemm(As[r], wts[r], Ss[r], outs[m], m, N_DIM, K_DIM, G_DIM)
+        if rc:
+            raise RuntimeError(w4.status_string(rc))
+
+    # warm the library's per-device setup outside any capture
+    launch(1, 0)
+    launch(16, 1)
+    torch.cuda.synchronize()
+
+    def capture(nsteps, start):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(nsteps):
+                launch(1, (2 * (start + i)) % R)
+                launch(16, (2 * (start + i) + 1) % R)
+        return g
+
+    K, W = args.steps, args.warmup
+    chunk = min(K, GRAPH_CHUNK)
+    g_main = capture(chunk, 0)
+    rem = K % chunk
+    g_rem = capture(rem, 0) if rem else None
+    for _ in range(max(1, math.ceil(W / chunk))):
+        g_main.replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    if rank == 0:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K // chunk):
+        g_main.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    e1.record()
+    e1.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    clocks = sampler.stop() if rank == 0 else None
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    sec = ms_max / 1e3
+    value = world * K * step_bytes() / sec / 1e9
+    tflops = world * K * step_flops() / sec / 1e12
+
+    status = w4.device_status(clear=True)
+    if status != w4.OK:
+        raise RuntimeError(f"device status after the timed region: {w4.status_string(status)}")
+
+    # End to end through the public API: pinned host activations in, results out, every step.
+    A1_h = torch.from_numpy(case.A[:1].copy()).pin_memory()
+    A16_h = torch.from_numpy(case.A.copy()).pin_memory()
+    C1_h = torch.empty((1, N_DIM), dtype=torch.float16).pin_memory()
+    C16_h = torch.empty((16, N_DIM), dtype=torch.float16).pin_memory()
+    A1_d = torch.empty((1, K_DIM), dtype=torch.float16, device=dev)
+    A16_d = torch.empty((16, K_DIM), dtype=torch.float16, device=dev)
+    K_e2e = min(K, 2000)
+
+    def e2e_step(i):
+        A1_d.copy_(A1_h, non_blocking=True)
+        A16_d.copy_(A16_h, non_blocking=True)
+        r1, r2 = (2 * i) % R, (2 * i + 1) % R
+        w4.gemm(A1_d, wts[r1], Ss[r1], N_DIM, G_DIM, out=C1)
+        w4.gemm(A16_d, wts[r2], Ss[r2], N_DIM, G_DIM, out=C16)
+        C1_h.copy_(C1, non_blocking=True)
+        C16_h.copy_(C16, non_blocking=True)
+
+    for i in range(20):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for i in range(K_e2e):
+        e2e_step(i)
+    f1.record()
+    f1.synchronize()
+    te = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_sec = float(te.item()) / 1e3
+    e2e = {"value": world * K_e2e * step_bytes() / e2e_sec / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": sum(m * K_DIM * 2 for m in M_STEP),
+           "d2h_bytes_per_step": sum(m * N_DIM * 2 for m in M_STEP), "steps": K_e2e}
+
+    extra = per_config(w4, dev) if (rank == 0 and not args.no_configs) else None
+    peaks = load_peaks()
+    achieved = K * step_bytes() / sec / 1e9  # per GPU: every launch in the step is the same kernel
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": list(M_STEP), "K": K_DIM, "N": N_DIM, "G": G_DIM,
+                   "l2": f"inputs larger than L2: {R} rotating copies of weights+scales+activations "
+                         f"({R * copy_bytes / 2 ** 20:.0f} MiB vs {l2 / 2 ** 20:.0f} MiB L2)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "tflops": round(tflops, 3),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic_from_profile(),
+                     "peak_source": f"{peaks['source']} (copy bandwidth)",
+                     "kernel": "w4a16_gemm_kernel<16,8,2,2> (token tile 16, K split over a cluster)"},
+        "e2e": e2e,
+        "gpu_launches": world * 2 * K,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        line["cpu_baseline"] = None if args.no_cpu_baseline else cpu_baseline()
+        if extra is not None:
+            line["per_config"] = extra
+        print(json.dumps(line), flush=True)
+    del g_main, g_rem
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def per_config(w4, dev):
+    """Device time per launch for every workload family (context for the headline line)."""
+    import torch
+    peaks = load_peaks()
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20)
+    out = {}
+    for name, cfg in workloads.CONFIGS.items():
+        if name == "tiny":
+            continue
+        c = workloads.make(name)
+        if cfg["kind"] == "dense":
+            _, wt = w4.prepare_weights(torch.from_numpy(c.q).to(dev))
+            S = torch.from_numpy(c.S).to(dev)
+            A = torch.from_numpy(c.A).to(dev)
+            C = torch.empty((c.M, c.N), dtype=torch.float16, device=dev)
+            per = wt.numel() + S.numel() * 2 + A.numel() * 2 + C.numel() * 2
+            R = max(2, math.ceil(2 * l2 / per) + 1)
+            bufs = [(wt, S, A, C)] + [(wt.clone(), S.clone(), A.clone(), torch.empty_like(C)) for _ in range(R - 1)]
+            M, N, K, G = c.M, c.N, c.K, c.G
+
+            def launch(r, b=bufs, M=M, N=N, K=K, G=G):
+                wt_, S_, A_, C_ = b[r]
+                rc = w4.w4a16_gemm(A_, wt_, S_, C_, M, N, K, G)
+                if rc:
+                    raise RuntimeError(w4.status_string(rc))
+            fl = flops(M, N, K)
+            by = algorithmic_bytes(M, N, K, G)
+        else:
+            wts = [w4.prepare_weights(torch.from_numpy(c.q[e]).to(dev))[1] for e in range(c.E)]
+            Ss = [torch.from_numpy(c.S[e]).to(dev) for e in range(c.E)]
+            A = torch.from_numpy(c.A).to(dev)
+            off = torch.from_numpy(c.offsets).to(dev)
+            C = torch.empty((c.total_rows, c.N), dtype=torch.float16, device=dev)
+            per = sum(x.numel() for x in wts) + sum(x.numel() * 2 for x in Ss)
+            R = max(2, math.ceil(2 * l2 / per) + 1)
+            sets = [(wts, Ss)] + [([x.clone() for x in wts], [x.clone() for x in Ss]) for _ in range(R - 1)]
+
+            def launch(r, sets=sets, A=A, off=off, C=C, c=c):
+                wts_, Ss_ = sets[r]
+                rc = w4.w4a16_grouped_gemm(A, wts_, Ss_, off, C, c.E, c.total_rows, c.N, c.K, c.G)
+                if rc:
+                    raise RuntimeError(w4.status_string(rc))
+            fl = flops(c.total_rows, c.N, c.K)
+            by = sum(algorithmic_bytes(int(c.offsets[e + 1] - c.offsets[e]), c.N, c.K, c.G) for e in range(c.E))
+        launch(0)
+        torch.cuda.synchronize()
+        n = 200 if fl < 1e10 else 40
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                launch(i % R)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / n
+        gbs = by / (us * 1e-6) / 1e9
+        tf = fl / (us * 1e-6) / 1e12
+        t_roof = max(by / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
+        out[name] = {"us_per_launch": round(us, 3), "GB/s": round(gbs, 1), "TFLOP/s": round(tf, 2),
+                     "roofline_frac": round(t_roof / (us * 1e-6), 4),
+                     "bound": "hbm" if by / (peaks["hbm_gbs"] * 1e9) >= fl / (peaks["bf16_tflops"] * 1e12)
+                     else "tensor", "rotating_copies": R}
+        del g
+    status = w4.device_status(clear=True)
+    if status != w4.OK:
+        raise RuntimeError(f"device status after per-config timing: {w4.status_string(status)}")
+    return out
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    o = oracle.load()
+    case = workloads.dense(16, K_DIM, N_DIM, G_DIM, seed=1)
+    K, W = args.steps, args.warmup
+    # Calibrate a column sample so that warm-up plus timed steps take about two minutes.
+    probe = oracle_sample(o, case, 64)
+    oracle_decode_step(o, case, probe)
+    t0 = time.perf_counter()
+    oracle_decode_step(o, case, probe)
+    t64 = max(time.perf_counter() - t0, 1e-6)
+    cols = int(64 * (120.0 / (K + W)) / t64)
+    cols = max(8, min(N_DIM, cols - cols % 8))
+    sample = oracle_sample(o, case, cols)
+    for _ in range(W):
+        oracle_decode_step(o, case, sample)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        oracle_decode_step(o, case, sample)
+    sec = time.perf_counter() - t0
+    value = K * sample_bytes(cols) / sec / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": sec * 1e3 / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "M": list(M_STEP), "K": K_DIM, "N": N_DIM, "G": G_DIM,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": o.threads(), "kind": "oracle",
+                         "sample": f"each step: M=1 and M=16 over the first {cols} of {N_DIM} columns "
+                                   f"(K=4096, G=128), fp64 oracle"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--warmup", type=int, default=1000)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-config timings")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,120 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point the
+header declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import weight_only_int4_wise_b200 as w
+from weight_only_int4_wise_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a16.h")
+
+FAKE = 0x10000  # a non-null, 16-byte aligned address that is never dereferenced on these paths
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(w4a16_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("w4a16_pack", "w4a16_unpack", "w4a16_repack", "w4a16_gemm", "w4a16_grouped_gemm",
+                     "w4a16_status_string", "w4a16_tiled_bytes", "w4a16_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in w4a16.h but not exported"
+    assert sorted(_lib.EXPORTED) == declared_functions()
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert w.status_string(code) != "unknown status"
+    assert w.status_string(99) == "unknown status"
+
+
+def test_tiled_bytes_matches_layout_definition(lib):
+    o = oracle.load()
+    for K, N in [(1, 1), (64, 128), (65, 129), (4096, 4096), (4096, 14336), (14336, 4096), (72, 200)]:
+        assert w.w4a16_tiled_bytes(K, N) == o.tiled_bytes(K, N)
+    assert w.w4a16_tiled_bytes(0, 5) == 0 and w.w4a16_tiled_bytes(5, -1) == 0
+
+
+def test_gemm_rejects_bad_arguments_on_host(lib):
+    g = lambda **kw: w.w4a16_gemm(kw.get("A", FAKE), kw.get("Wt", FAKE), kw.get("S", FAKE), kw.get("C", FAKE),
+                                  kw.get("M", 4), kw.get("N", 128), kw.get("K", 128), kw.get("G", 64), stream=0)
+    assert g(A=None) == w.ERR_INVALID_ARG
+    assert g(Wt=None) == w.ERR_INVALID_ARG
+    assert g(C=None) == w.ERR_INVALID_ARG
+    assert g(M=-1) == w.ERR_INVALID_ARG
+    assert g(N=0) == w.ERR_INVALID_ARG
+    assert g(K=0) == w.ERR_INVALID_ARG
+    assert g(G=0) == w.ERR_INVALID_ARG
+    assert g(N=100) == w.ERR_UNSUPPORTED   # N % 8
+    assert g(K=100) == w.ERR_UNSUPPORTED   # K % 8
+    assert g(G=24) == w.ERR_UNSUPPORTED    # G % 16
+    assert g(A=FAKE + 8) == w.ERR_MISALIGNED
+    assert g(Wt=FAKE + 4) == w.ERR_MISALIGNED
+    assert g(S=FAKE + 2) == w.ERR_MISALIGNED
+    assert g(C=FAKE + 1) == w.ERR_MISALIGNED
+    assert g(M=0) == w.OK  # empty batch: nothing to do, nothing launched
+
+
+def test_grouped_rejects_bad_arguments_on_host(lib):
+    def g(E=2, rows=8, wts=None, ss=None, off=FAKE, A=FAKE, C=FAKE, N=128, K=128, G=64):
+        wts = [FAKE] * E if wts is None else wts
+        ss = [FAKE] * E if ss is None else ss
+        return w.w4a16_grouped_gemm(A, wts, ss, off, C, E, rows, N, K, G, stream=0)
+    assert g(E=0, wts=[FAKE], ss=[FAKE]) == w.ERR_INVALID_ARG
+    assert g(E=w.MAX_EXPERTS + 1) == w.ERR_INVALID_ARG
+    assert g(off=None) == w.ERR_INVALID_ARG
+    assert g(rows=-1) == w.ERR_INVALID_ARG
+    assert g(wts=[FAKE, 0]) == w.ERR_INVALID_ARG
+    assert g(wts=[FAKE, FAKE + 8]) == w.ERR_MISALIGNED
+    assert g(off=FAKE + 2) == w.ERR_MISALIGNED
+    assert g(G=40) == w.ERR_UNSUPPORTED
+    assert g(rows=0) == w.OK
+
+
+def test_pack_rejects_bad_arguments_on_host(lib):
+    assert w.w4a16_pack(None, FAKE, 4, 4, stream=0) == w.ERR_INVALID_ARG
+    assert w.w4a16_pack(FAKE, FAKE, 0, 4, stream=0) == w.ERR_INVALID_ARG
+    assert w.w4a16_unpack(FAKE, None, 4, 4, stream=0) == w.ERR_INVALID_ARG
+    assert w.w4a16_repack(FAKE, FAKE + 4, 4, 4, stream=0) == w.ERR_MISALIGNED
+    assert w.w4a16_repack(FAKE, FAKE, 4, -4, stream=0) == w.ERR_INVALID_ARG
+
+
+def test_launch_plan_on_host(lib):
+    # Nominal plans (no device here): decode splits K across a cluster; prefill tiles M.
+    rc, info = w.w4a16_gemm_launch_info(1, 4096, 4096, 128)
+    assert rc == w.OK and info.token_tile == 16 and info.k_splits > 1 and info.grid_y == 32
+    rc, info = w.w4a16_gemm_launch_info(2048, 4096, 4096, 128)
+    assert rc == w.OK and info.token_tile == 256 and info.k_splits == 1 and info.grid_z == 8
+    rc, info = w.w4a16_grouped_launch_info(8, 1024, 14336, 4096, 128)
+    assert rc == w.OK and info.grid_y == 112 and info.grid_z >= 8
+    rc, _ = w.w4a16_gemm_launch_info(0, 4096, 4096, 128)
+    assert rc == w.ERR_INVALID_ARG
+
+
+def test_valid_call_without_a_gpu_is_refused_not_crashed(lib):
+    try:
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("a GPU is present")
+    except ImportError:
+        pass
+    rc = w.w4a16_gemm(FAKE, FAKE, FAKE, FAKE, 4, 128, 128, 64, stream=0)
+    assert rc == w.ERR_UNSUPPORTED

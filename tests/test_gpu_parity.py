@@ -1,0 +1,228 @@
+"""CUDA path against the CPU oracle on the same seeded inputs, through the C ABI.
+
+Integer work (pack, unpack, repack) must be bit-exact; the GEMM must satisfy
+|gpu - ref| <= 1e-2 + 5e-3 * |ref| element by element. Small cases are compared
+in full; the full-size workloads in the launch configuration the benchmark uses
+are compared in full where the oracle is quick and on sampled elements
+otherwise."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import pins
+import workloads
+import weight_only_int4_wise_b200 as w
+from gpu_util import dev, device_weights, guarded_output, guards_intact, within_tolerance
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def o():
+    return oracle.load()
+
+
+@pytest.fixture(autouse=True)
+def clean_status():
+    w.device_status(clear=True)
+    yield
+    assert w.device_status(clear=True) == w.OK
+
+
+# ------------------------------------------------------------------ packing
+
+@pytest.mark.parametrize("K,N", [(1, 8), (7, 24), (512, 512), (4096, 4096), (4095, 136)])
+def test_pack_bit_exact(o, K, N):
+    q = workloads.dense(1, K, N, 16, seed=K + N).q
+    wp = w.pack(dev(q))
+    torch.cuda.synchronize()
+    assert np.array_equal(wp.cpu().numpy(), o.pack(q))
+    assert np.array_equal(w.unpack(wp, K).cpu().numpy(), q)
+
+
+def test_pack_all_byte_values(o):
+    wp = torch.arange(256, dtype=torch.uint8, device="cuda").view(1, 256)
+    q = w.unpack(wp, 2)
+    assert np.array_equal(q.cpu().numpy(), o.unpack(wp.cpu().numpy(), 2))
+    assert np.array_equal(w.pack(q).cpu().numpy(), wp.cpu().numpy())
+
+
+@pytest.mark.parametrize("K,N", [(64, 128), (72, 136), (200, 520), (4096, 4096), (4100, 264)])
+def test_repack_bit_exact(o, K, N):
+    q = workloads.dense(1, K, N, 16, seed=3 * K + N).q
+    _, wt = device_weights(q)
+    torch.cuda.synchronize()
+    assert np.array_equal(wt.cpu().numpy(), o.tile(q))
+
+
+# --------------------------------------------------------------- small GEMMs
+
+def run_dense(o, M, K, N, G, seed, a_scale=1.0):
+    c = workloads.dense(M, K, N, G, seed, a_scale=a_scale)
+    _, wt = device_weights(c.q)
+    flat, C, pad = guarded_output(M, N)
+    w.gemm(dev(c.A), wt, dev(c.S), N, G, out=C)
+    torch.cuda.synchronize()
+    got = C.cpu().numpy()
+    ref = o.gemm(c.A, pins.python_pack(c.q), c.S, K, G)
+    ok, err, rel = within_tolerance(got, ref)
+    assert ok, f"M={M} K={K} N={N} G={G}: max abs err {err}, max rel err {rel}"
+    assert guards_intact(flat, pad, M * N), "the kernel wrote outside C"
+    return got, ref
+
+
+def test_tiny_config(o):
+    cfg = workloads.CONFIGS["tiny"]
+    run_dense(o, cfg["M"], cfg["K"], cfg["N"], cfg["G"], cfg["seed"])
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 16, 17, 33, 64, 65, 127, 129, 200, 256, 257, 300])
+def test_ragged_rows(o, M):
+    # several column tiles with a ragged last one, several K stages, every token-tile size
+    run_dense(o, M, 200, 392, 64, seed=100 + M)
+
+
+@pytest.mark.parametrize("K,N,G", [
+    (64, 8, 64), (72, 136, 16), (96, 128, 32), (208, 264, 48), (200, 520, 80), (520, 256, 128),
+    (512, 384, 512), (256, 128, 4096), (1024, 256, 64), (1032, 136, 16),
+])
+def test_shapes_and_group_sizes(o, K, N, G):
+    for M in (1, 8, 40):
+        run_dense(o, M, K, N, G, seed=K * 7 + N + G + M)
+
+
+def test_large_activations_stay_in_tolerance(o):
+    # |A| ~ 8: outputs of tens of units exercise the relative part of the bound
+    run_dense(o, 16, 2048, 256, 128, seed=77, a_scale=8.0)
+
+
+def test_deterministic(o):
+    c = workloads.dense(5, 4096, 512, 128, 5)
+    _, wt = device_weights(c.q)
+    A, S = dev(c.A), dev(c.S)
+    r1 = w.gemm(A, wt, S, 512, 128).cpu().numpy()
+    r2 = w.gemm(A, wt, S, 512, 128).cpu().numpy()
+    assert np.array_equal(r1.view(np.uint16), r2.view(np.uint16))
+
+
+# --------------------------------------------------------------- grouped
+
+def run_grouped(o, case):
+    _ = [device_weights(case.q[e]) for e in range(case.E)]
+    wts = [x[1] for x in _]
+    Ss = [dev(case.S[e]) for e in range(case.E)]
+    flat, C, pad = guarded_output(case.total_rows, case.N)
+    w.grouped_gemm(dev(case.A), wts, Ss, dev(case.offsets), case.N, case.G, out=C)
+    torch.cuda.synchronize()
+    got = C.cpu().numpy()
+    ref = o.grouped_gemm(case.A, [pins.python_pack(case.q[e]) for e in range(case.E)], list(case.S),
+                         case.offsets, case.K, case.G)
+    ok, err, rel = within_tolerance(got, ref)
+    assert ok, f"grouped: max abs err {err}, max rel err {rel}"
+    assert guards_intact(flat, pad, case.total_rows * case.N)
+    return got, ref
+
+
+def test_grouped_small_with_empty_expert(o):
+    run_grouped(o, workloads.grouped(E=6, top_k=2, tokens=100, K=256, N=392, G=64, seed=31, empty_experts=[1, 4]))
+
+
+def test_grouped_uneven_segments(o):
+    # 300 tokens routed top-1 over 3 experts: segments of about 100 rows, several token tiles
+    run_grouped(o, workloads.grouped(E=3, top_k=1, tokens=300, K=512, N=256, G=128, seed=32))
+
+
+def test_grouped_single_expert_equals_dense(o):
+    c = workloads.dense(70, 512, 256, 128, 33)
+    _, wt = device_weights(c.q)
+    A, S = dev(c.A), dev(c.S)
+    dense = w.gemm(A, wt, S, 256, 128)
+    off = torch.tensor([0, 70], dtype=torch.int32, device="cuda")
+    grouped = w.grouped_gemm(A, [wt], [S], off, 256, 128)
+    torch.cuda.synchronize()
+    ok, err, _ = within_tolerance(grouped.cpu().numpy(), dense.cpu().numpy())
+    assert ok, err
+
+
+def test_grouped_rejects_malformed_offsets_on_device():
+    c = workloads.dense(8, 128, 128, 64, 34)
+    _, wt = device_weights(c.q)
+    A, S = dev(c.A), dev(c.S)
+    for bad in ([0, 5, 3], [1, 4, 8], [0, 4, 7]):  # decreasing, nonzero start, wrong end
+        flat, C, pad = guarded_output(8, 128)
+        w.grouped_gemm(A, [wt, wt], [S, S], torch.tensor(bad, dtype=torch.int32, device="cuda"), 128, 64, out=C)
+        assert w.device_status(clear=True) == w.ERR_BAD_OFFSETS
+        assert guards_intact(flat, pad, 0) and np.all(C.cpu().numpy().view(np.uint16) == 0x7BAD)
+
+
+def test_misaligned_pointer_is_refused():
+    c = workloads.dense(4, 128, 128, 64, 35)
+    _, wt = device_weights(c.q)
+    A = dev(c.A)
+    buf = torch.empty(4 * 128 + 8, dtype=torch.float16, device="cuda")
+    rc = w.w4a16_gemm(A.data_ptr() + 2, wt, dev(c.S), buf, 4, 128, 128, 64)
+    assert rc == w.ERR_MISALIGNED
+
+
+# ------------------------------------------------- full-size workloads
+
+DENSE_FULL = ["decode_m1", "decode_m16", "mlp_up", "mlp_down", "mlp_up_g64"]
+
+
+@pytest.mark.parametrize("name", DENSE_FULL)
+def test_full_size_skinny_configs(o, name):
+    c = workloads.make(name)
+    _, wt = device_weights(c.q)
+    flat, C, pad = guarded_output(c.M, c.N)
+    w.gemm(dev(c.A), wt, dev(c.S), c.N, c.G, out=C)
+    torch.cuda.synchronize()
+    got = C.cpu().numpy()
+    ref = o.gemm(c.A, pins.python_pack(c.q), c.S, c.K, c.G)
+    ok, err, rel = within_tolerance(got, ref)
+    assert ok, f"{name}: max abs err {err}, max rel err {rel}"
+    assert guards_intact(flat, pad, c.M * c.N)
+
+
+def sample_positions(M, N, count, seed):
+    g = np.random.Generator(np.random.PCG64(seed))
+    rows = list(g.integers(0, M, size=count)) + [0, M - 1] * 64 + list(range(0, M, max(1, M // 64)))
+    cols = list(g.integers(0, N, size=count)) + list(range(0, 128)) + [N - 1] * (len(range(0, M, max(1, M // 64))))
+    return np.array(rows, dtype=np.int64), np.array(cols, dtype=np.int64)
+
+
+def test_full_size_prefill_sampled(o):
+    c = workloads.make("prefill")
+    _, wt = device_weights(c.q)
+    flat, C, pad = guarded_output(c.M, c.N)
+    w.gemm(dev(c.A), wt, dev(c.S), c.N, c.G, out=C)
+    torch.cuda.synchronize()
+    got = C.cpu().numpy()
+    assert guards_intact(flat, pad, c.M * c.N)
+    assert np.all(np.isfinite(got))
+    rows, cols = sample_positions(c.M, c.N, 3000, 41)
+    ref = o.gemm_sample(c.A, pins.python_pack(c.q), c.S, c.K, c.G, rows, cols)
+    ok, err, rel = within_tolerance(got[rows, cols], ref)
+    assert ok, f"prefill: max abs err {err}, max rel err {rel}"
+
+
+def test_full_size_grouped_sampled(o):
+    c = workloads.make("grouped")
+    wts = [device_weights(c.q[e])[1] for e in range(c.E)]
+    Ss = [dev(c.S[e]) for e in range(c.E)]
+    flat, C, pad = guarded_output(c.total_rows, c.N)
+    w.grouped_gemm(dev(c.A), wts, Ss, dev(c.offsets), c.N, c.G, out=C)
+    torch.cuda.synchronize()
+    got = C.cpu().numpy()
+    assert guards_intact(flat, pad, c.total_rows * c.N)
+    assert np.all(np.isfinite(got))
+    g = np.random.Generator(np.random.PCG64(42))
+    for e in range(c.E):
+        r0, r1 = int(c.offsets[e]), int(c.offsets[e + 1])
+        if r1 == r0:
+            continue
+        rows = np.concatenate([g.integers(0, r1 - r0, size=300), [0, r1 - r0 - 1]]).astype(np.int64)
+        cols = np.concatenate([g.integers(0, c.N, size=300), [c.N - 1, 0]]).astype(np.int64)
+        ref = o.gemm_sample(c.A[r0:r1], pins.python_pack(c.q[e]), c.S[e], c.K, c.G, rows, cols)
+        ok, err, rel = within_tolerance(got[r0 + rows, cols], ref)
+        assert ok, f"grouped expert {e}: max abs err {err}, max rel err {rel}"

@@ -1,0 +1,845 @@
+// W4A16 group-wise GEMM on sm_100a: C[M,N] = A[M,K] x dequant(W)[K,N].
+//
+// The operation is the one the Int4GroupwiseGemmPluginV2 page describes
+// (class description: activations [b,seq,K] fp16, int4 weights, scales
+// [ceil(K/G),N] fp16, output [b,seq,N] fp16; constructor: N columns, K rows,
+// groupSize G). The grouped-expert entry point applies it per expert segment
+// of gathered rows (Int4MoePlugin page, constructor parameters).
+//
+// One kernel template serves decode (M = 1..16), skinny, prefill and
+// grouped-expert shapes. It computes the transposed product
+//     D[n, m] = sum_k W[k, n] * A[m, k]
+// on the 5th-generation tensor core: each CTA owns 128 weight columns (the MMA
+// M extent, one TMEM lane per column) and a tile of BN activation rows (the
+// MMA N extent, 16..256), so that small token counts cost no padding of the
+// weight side. Warp roles inside a CTA (320 threads):
+//   warp 0      producer: per 64-deep K stage, one TMA tile load of the
+//               activations (128-byte swizzle, zero fill past M and K), one
+//               4096-byte bulk copy of the tiled int4 weights and the scale rows.
+//   warp 1      TMEM allocation and the single MMA-issuing thread
+//               (tcgen05.mma kind::f16, fp32 accumulator in TMEM).
+//   warps 2..9  dequantisation: each thread turns 32 int4 codes of one column
+//               into fp16 (magic-exponent decode, times the group scale) and
+//               stores them into the K-major swizzled A-operand tile; then the
+//               epilogue (tcgen05.ld -> fp16 -> global).
+// Small-M shapes split K across up to 8 CTAs of one thread-block cluster; the
+// fp32 partial tiles are summed in rank order through distributed shared
+// memory (deterministic, no global workspace).
+//
+// Every wait is bounded: a wait that runs out latches W4A16_ERR_TIMEOUT in the
+// device status word, and the CTA drains its copies, frees its TMEM and exits.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/w4a16.h"
+#include "ptx.cuh"
+#include "w4a16_internal.h"
+
+namespace w4a16 {
+
+__device__ int g_status;  // latched device-side error (0 = none)
+
+constexpr int kTileN = 128;                 // weight columns per CTA (MMA M)
+constexpr int kTileK = 64;                  // K per pipeline stage
+constexpr int kRawBytes = 4096;             // int4 codes of one 128 x 64 tile
+constexpr int kW16Bytes = kTileN * kTileK * 2;  // dequantised fp16 tile
+constexpr int kMaxScaleRows = 4;            // scale rows one stage can touch (G >= 16)
+constexpr int kScaleRowBytes = kTileN * 2;
+constexpr int kDequantWarps = 8;
+constexpr int kThreads = (2 + kDequantWarps) * 32;
+constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per wait
+
+struct Params {
+    const uint8_t* wt[W4A16_MAX_EXPERTS];   // tiled weights (dense: [0])
+    const __half* sc[W4A16_MAX_EXPERTS];    // scales [ceil(K/G), N]
+    const int32_t* offsets;                 // grouped: [E+1] on the device
+    __half* C;
+    int32_t rows;       // dense: M; grouped: total gathered rows
+    int32_t N, K, G;
+    int32_t ngroups;    // ceil(K/G)
+    int32_t KT;         // ceil(K/64)
+    int32_t E;          // grouped: number of experts; dense: 1
+    int32_t splits;     // CTAs along K (cluster size along x)
+    int32_t scale_rows; // scale rows fetched per stage
+    int32_t scale_mode; // 0: G % 64 == 0, 1: G == 32, 2: G == 16, 3: other
+    int32_t grouped;
+};
+
+template <int BN, int LS, int WS>
+struct Layout {
+    static constexpr int kActBytes = BN * 128;
+    static constexpr int kAct = 0;
+    static constexpr int kW16 = kAct + LS * kActBytes;
+    static constexpr int kRaw = kW16 + WS * kW16Bytes;
+    static constexpr int kScale = kRaw + LS * kRawBytes;
+    static constexpr int kInfo = kScale + LS * kMaxScaleRows * kScaleRowBytes;  // int2 per stage
+    static constexpr int kBar = kInfo + LS * 8;
+    static constexpr int kNumBars = 2 * LS + 2 * WS + 1;
+    static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base, abort flag, tile info
+    static constexpr int kTotal = kMisc + 32;
+    static constexpr int kAlloc = kTotal + 1024;       // slack for aligning the base to 1024
+    static constexpr int kTmemCols = BN < 32 ? 32 : BN;
+    static constexpr int kRedBytes = BN * kTileN * 4;  // split-K partials, alias the operand rings
+    static_assert(kRedBytes <= kW16 + WS * kW16Bytes, "split-K buffer must fit in the operand rings");
+    static_assert((kActBytes % 1024) == 0 && (kW16 % 1024) == 0, "operand tiles need 1024-byte alignment");
+};
+
+__device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
+
+// Bounded wait on an mbarrier phase. Returns false if the CTA is aborting or
+// the wait ran out (which starts the abort).
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kTimeoutNs) {
+                *abort_flag = 1;
+                latch_status(W4A16_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded wait that ignores the abort flag: used where in-flight asynchronous
+// work must finish before its resources are released.
+__device__ __forceinline__ bool drain_phase(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 63u && global_timer_ns() - t0 > kTimeoutNs) {
+            latch_status(W4A16_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Warp-collective forms: lane 0 polls (so the timeout decision is the same for
+// the whole warp), then every lane observes the completed phase itself, which
+// gives each lane acquire ordering on the data the phase guards. The phase
+// cannot move on before this warp arrives elsewhere, so that check is immediate.
+__device__ __forceinline__ bool warp_wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_phase(bar, parity, abort_flag) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) mbar_try_wait(bar, parity);
+    return ok != 0;
+}
+
+__device__ __forceinline__ void warp_drain_phase(uint64_t* bar, uint32_t parity) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = drain_phase(bar, parity) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) mbar_try_wait(bar, parity);
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
+
+// Eight int4 codes of one word (nibble i = k_local {0,2,4,6,1,3,5,7}[i]) ->
+// eight fp16 weights q*s in natural k order. Each code c is read as the fp16
+// number 1024 + (c ^ 8) (or 1024 + 16*(c ^ 8) for the high nibble of a byte)
+// by OR-ing it under the exponent of 1024; subtracting the bias then gives the
+// signed code exactly, and one multiply applies the group scale.
+__device__ __forceinline__ uint4 dequant_word(uint32_t x, __half2 s2) {
+    const __half2 bias_lo = bits_h2(0x64086408u);  // 1032, 1032
+    const __half2 sixteenth = bits_h2(0x2C002C00u);  // 1/16, 1/16
+    const __half2 bias_hi = bits_h2(0xD480D480u);  // -72, -72
+    const uint32_t b0 = lop3_and_xor(x, 0x000F000Fu, 0x64086408u);
+    const uint32_t t0 = lop3_and_xor(x, 0x00F000F0u, 0x64806480u);
+    const uint32_t x8 = x >> 8;
+    const uint32_t b1 = lop3_and_xor(x8, 0x000F000Fu, 0x64086408u);
+    const uint32_t t1 = lop3_and_xor(x8, 0x00F000F0u, 0x64806480u);
+    const __half2 q01 = __hsub2(bits_h2(b0), bias_lo);
+    const __half2 q23 = __hfma2(bits_h2(t0), sixteenth, bias_hi);
+    const __half2 q45 = __hsub2(bits_h2(b1), bias_lo);
+    const __half2 q67 = __hfma2(bits_h2(t1), sixteenth, bias_hi);
+    uint4 out;
+    out.x = h2_bits(__hmul2(q01, s2));
+    out.y = h2_bits(__hmul2(q23, s2));
+    out.z = h2_bits(__hmul2(q45, s2));
+    out.w = h2_bits(__hmul2(q67, s2));
+    return out;
+}
+
+template <int BN, int LS, int WS, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB)
+    w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ Params p) {
+    using L = Layout<BN, LS, WS>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base_addr = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (base_addr & 1023u)) & 1023u);
+
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
+    uint64_t* empty = full + LS;
+    uint64_t* wfull = empty + LS;
+    uint64_t* wempty = wfull + WS;
+    uint64_t* accfull = wempty + WS;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    int* tile_info = reinterpret_cast<int*>(smem + L::kMisc + 8);  // has_tile, expert, m0, rows
+    int2* stage_info = reinterpret_cast<int2*>(smem + L::kInfo);    // {first scale row, rows valid}
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nt = blockIdx.y;
+
+    // ---------------------------------------------------------------- tile
+    if (threadIdx.x == 0) {
+        int has = 1, expert = 0, m0 = 0, rows = 0;
+        if (p.grouped) {
+            const int32_t* off = p.offsets;
+            bool ok = off[0] == 0 && off[p.E] == p.rows;
+            for (int e = 0; e < p.E && ok; ++e) ok = off[e + 1] >= off[e];
+            has = 0;
+            if (!ok) {
+                latch_status(W4A16_ERR_BAD_OFFSETS);
+            } else {
+                int z = blockIdx.z;
+                for (int e = 0; e < p.E; ++e) {
+                    const int cnt = off[e + 1] - off[e];
+                    const int tiles = (cnt + BN - 1) / BN;
+                    if (z < tiles) {
+                        has = 1;
+                        expert = e;
+                        m0 = off[e] + z * BN;
+                        rows = min(BN, off[e + 1] - m0);
+                        break;
+                    }
+                    z -= tiles;
+                }
+            }
+        } else {
+            m0 = blockIdx.z * BN;
+            rows = min(BN, p.rows - m0);
+        }
+        tile_info[0] = has;
+        tile_info[1] = expert;
+        tile_info[2] = m0;
+        tile_info[3] = rows;
+    }
+    __syncthreads();
+    if (!tile_info[0]) return;  // grouped slot beyond the routed tiles (no cluster in that mode)
+    const int expert = tile_info[1];
+    const int m0 = tile_info[2];
+    const int rows = tile_info[3];
+    const int split = p.grouped ? 0 : static_cast<int>(blockIdx.x);
+    const int kb = static_cast<int>((static_cast<int64_t>(split) * p.KT) / p.splits);
+    const int ke = static_cast<int>((static_cast<int64_t>(split + 1) * p.KT) / p.splits);
+    const int nst = ke - kb;
+    const int n_mma = min(BN, (rows + 15) & ~15);
+    const uint32_t idesc = idesc_f16_f32(128, static_cast<uint32_t>(n_mma));
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < LS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1 + kDequantWarps);
+        }
+        for (int w = 0; w < WS; ++w) {
+            mbar_init(&wfull[w], kDequantWarps);
+            mbar_init(&wempty[w], 1);
+        }
+        mbar_init(accfull, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensor_map(&tmA);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, L::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_acc = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint8_t* wsrc = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes;
+            const __half* ssrc = p.sc[expert] + static_cast<int64_t>(nt) * kTileN;
+            const int ncols = min(kTileN, p.N - nt * kTileN);
+            const uint32_t srow_bytes = static_cast<uint32_t>(ncols) * 2u;
+            int issued = 0;
+            for (int i = 0; i < nst; ++i) {
+                const int s = i % LS;
+                if (i >= LS && !wait_phase(&empty[s], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
+                    break;
+                const int kt = kb + i;
+                const int g0 = (kt * kTileK) / p.G;
+                const int nrows = min(p.scale_rows, p.ngroups - g0);
+                stage_info[s] = make_int2(g0, nrows);
+                const uint32_t bytes = static_cast<uint32_t>(L::kActBytes + kRawBytes) + nrows * srow_bytes;
+                mbar_arrive_expect_tx(&full[s], bytes);
+                tma_load_2d(smem + L::kAct + s * L::kActBytes, &tmA, kt * kTileK, m0, &full[s]);
+                bulk_g2s(smem + L::kRaw + s * kRawBytes, wsrc + static_cast<int64_t>(kt) * kRawBytes, kRawBytes,
+                         &full[s]);
+                for (int r = 0; r < nrows; ++r)
+                    bulk_g2s(smem + L::kScale + (s * kMaxScaleRows + r) * kScaleRowBytes,
+                             ssrc + static_cast<int64_t>(g0 + r) * p.N, srow_bytes, &full[s]);
+                issued = i + 1;
+            }
+            // Every issued copy must land before the CTA's shared memory is released.
+            for (int i = max(0, issued - LS); i < issued; ++i)
+                drain_phase(&full[i % LS], static_cast<uint32_t>(i / LS) & 1u);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            for (int i = 0; i < nst; ++i) {
+                const int s = i % LS;
+                const int w = i % WS;
+                if (!wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
+                if (!wait_phase(&wfull[w], static_cast<uint32_t>(i / WS) & 1u, abort_flag)) break;
+                tc_fence_after_sync();
+                const uint32_t a0 = smem_addr(smem + L::kW16 + w * kW16Bytes);
+                const uint32_t b0 = smem_addr(smem + L::kAct + s * L::kActBytes);
+#pragma unroll
+                for (int kk = 0; kk < kTileK / 16; ++kk) {
+                    mma_f16_ss(tmem_acc, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
+                               (i | kk) != 0 ? 1u : 0u);
+                }
+                mma_commit(&empty[s]);
+                mma_commit(&wempty[w]);
+            }
+            mma_commit(accfull);  // fires once every MMA issued above has completed
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ dequant + epilogue
+        const int dw = warp - 2;
+        const int h = dw >> 2;            // which 32-deep half of the stage
+        const int quad = warp & 3;        // TMEM lane quadrant this warp may access
+        const int j = quad * 32 + lane;   // weight column inside the tile
+        const int n = nt * kTileN + j;
+        const bool col_ok = n < p.N;
+        for (int i = 0; i < nst; ++i) {
+            const int s = i % LS;
+            const int w = i % WS;
+            if (!warp_wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
+            const uint4 raw =
+                *reinterpret_cast<const uint4*>(smem + L::kRaw + s * kRawBytes + h * 2048 + j * 16);
+            const int2 info = stage_info[s];
+            const __half* srow = reinterpret_cast<const __half*>(smem + L::kScale + s * kMaxScaleRows * kScaleRowBytes);
+            const int last = info.y - 1;
+            __half sv[4];
+            if (p.scale_mode == 0) {
+                const __half v = srow[j];
+                sv[0] = sv[1] = sv[2] = sv[3] = v;
+            } else if (p.scale_mode == 1) {
+                const __half v = srow[min(h, last) * kTileN + j];
+                sv[0] = sv[1] = sv[2] = sv[3] = v;
+            } else if (p.scale_mode == 2) {
+                const __half v0 = srow[min(2 * h, last) * kTileN + j];
+                const __half v1 = srow[min(2 * h + 1, last) * kTileN + j];
+                sv[0] = sv[1] = v0;
+                sv[2] = sv[3] = v1;
+            } else {
+                const int k0 = (kb + i) * kTileK + 32 * h;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) sv[q] = srow[min((k0 + 8 * q) / p.G - info.x, last) * kTileN + j];
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+
+            uint4 o0 = dequant_word(raw.x, __half2half2(sv[0]));
+            uint4 o1 = dequant_word(raw.y, __half2half2(sv[1]));
+            uint4 o2 = dequant_word(raw.z, __half2half2(sv[2]));
+            uint4 o3 = dequant_word(raw.w, __half2half2(sv[3]));
+            if (!col_ok) o0 = o1 = o2 = o3 = make_uint4(0, 0, 0, 0);
+
+            if (i >= WS && !warp_wait_phase(&wempty[w], static_cast<uint32_t>((i / WS) - 1) & 1u, abort_flag))
+                break;
+            uint8_t* row = smem + L::kW16 + w * kW16Bytes + j * 128;
+            const int sw = j & 7;
+            *reinterpret_cast<uint4*>(row + (((4 * h + 0) ^ sw) << 4)) = o0;
+            *reinterpret_cast<uint4*>(row + (((4 * h + 1) ^ sw) << 4)) = o1;
+            *reinterpret_cast<uint4*>(row + (((4 * h + 2) ^ sw) << 4)) = o2;
+            *reinterpret_cast<uint4*>(row + (((4 * h + 3) ^ sw) << 4)) = o3;
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&wfull[w]);
+        }
+
+        // -------------------------------------------------- epilogue
+        // The accumulator is complete (or the CTA is aborting) once accfull fires;
+        // either way no MMA may still run when TMEM is released.
+        warp_drain_phase(accfull, 0);
+        tc_fence_after_sync();
+        const int aborted = __shfl_sync(0xffffffffu, *abort_flag, 0);
+        const bool have_acc = !aborted && nst > 0;
+        const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
+        if (p.splits == 1) {
+            if (have_acc) {
+                __half* cbase = p.C + static_cast<int64_t>(m0) * p.N + n;
+                for (int c = h; c < n_mma / 16; c += 2) {
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(tmem_acc + tlane + c * 16, v);
+                    tmem_ld_wait();
+                    if (col_ok) {
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) {
+                            const int r = c * 16 + t;
+                            if (r < rows) cbase[static_cast<int64_t>(r) * p.N] = __float2half_rn(__uint_as_float(v[t]));
+                        }
+                    }
+                }
+            }
+        } else {
+            float* red = reinterpret_cast<float*>(smem + L::kAct);
+            for (int c = h; c < BN / 16; c += 2) {
+                uint32_t v[16];
+                if (have_acc && c * 16 < n_mma) {
+                    tmem_ld_32x32b_x16(tmem_acc + tlane + c * 16, v);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) v[t] = 0u;
+                }
+#pragma unroll
+                for (int t = 0; t < 16; ++t) red[(c * 16 + t) * kTileN + j] = __uint_as_float(v[t]);
+            }
+        }
+        tc_fence_before_sync();
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_acc, L::kTmemCols);
+    }
+
+    if (p.splits > 1) {
+        // Sum the cluster's partial tiles in rank order; rank r writes columns
+        // [r*128/S, (r+1)*128/S) of the tile.
+        cluster_sync_all();
+        const int S = p.splits;
+        const int cw = kTileN / S;
+        const int rank = static_cast<int>(cluster_ctarank());
+        const float* red = reinterpret_cast<const float*>(smem + L::kAct);
+        const bool aborted = *abort_flag != 0;
+        for (int o = threadIdx.x; o < cw * rows; o += kThreads) {
+            const int col = rank * cw + (o % cw);
+            const int tok = o / cw;
+            const int nn = nt * kTileN + col;
+            if (nn < p.N && !aborted) {
+                float acc = 0.f;
+                for (int src = 0; src < S; ++src) acc += ld_dsmem_f32(&red[tok * kTileN + col], static_cast<uint32_t>(src));
+                p.C[static_cast<int64_t>(m0 + tok) * p.N + nn] = __float2half_rn(acc);
+            }
+        }
+        cluster_sync_all();
+    }
+}
+
+// ====================================================================== host
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+struct Variant {
+    int bn;
+    int nominal_per_sm;  // the residency the variant is sized for (used when no device is present)
+    int smem;
+    const void* fn;
+    int (*launch)(const CUtensorMap&, const Params&, dim3, int, int, cudaStream_t);
+};
+
+template <int BN, int LS, int WS, int MINB>
+int launch_variant(const CUtensorMap& map, const Params& p, dim3 grid, int cluster_x, int smem, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    cfg.numAttrs = 0;
+    if (cluster_x > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, w4a16_gemm_kernel<BN, LS, WS, MINB>, map, p);
+    return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+template <int BN, int LS, int WS, int MINB>
+Variant make_variant() {
+    return Variant{BN, MINB, Layout<BN, LS, WS>::kAlloc, reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, WS, MINB>),
+                   &launch_variant<BN, LS, WS, MINB>};
+}
+
+// Token tiles and their pipeline depths: small tiles keep two CTAs per SM.
+const Variant kVariants[] = {
+    make_variant<16, 8, 2, 2>(),  make_variant<32, 8, 2, 2>(),  make_variant<64, 5, 2, 2>(),
+    make_variant<128, 5, 2, 1>(), make_variant<256, 4, 2, 1>(),
+};
+
+const Variant& variant_for(int bn) {
+    for (const Variant& v : kVariants)
+        if (v.bn == bn) return v;
+    return kVariants[4];
+}
+
+struct DeviceState {
+    bool ready = false;
+    int ctas_per_sm[5] = {0, 0, 0, 0, 0};
+};
+
+int prepare_device(DeviceState** out) {
+    static DeviceState states[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return W4A16_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    DeviceState& st = states[dev];
+    if (!st.ready) {
+        for (int i = 0; i < 5; ++i) {
+            const Variant& v = kVariants[i];
+            if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess)
+                return W4A16_ERR_CUDA;
+            int n = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, v.fn, kThreads, v.smem) != cudaSuccess || n < 1)
+                return W4A16_ERR_CUDA;
+            // Every resident CTA holds TMEM columns; never ask for more than the SM has.
+            const int cols = v.bn < 32 ? 32 : v.bn;
+            if (n * cols > 512) n = 512 / cols;
+            st.ctas_per_sm[i] = n;
+        }
+        st.ready = true;
+    }
+    *out = &st;
+    return W4A16_OK;
+}
+
+int variant_index(int bn) {
+    for (int i = 0; i < 5; ++i)
+        if (kVariants[i].bn == bn) return i;
+    return 4;
+}
+
+int token_tile_for(int64_t rows_per_tile) {
+    if (rows_per_tile <= 16) return 16;
+    if (rows_per_tile <= 32) return 32;
+    if (rows_per_tile <= 64) return 64;
+    if (rows_per_tile <= 128) return 128;
+    return 256;
+}
+
+int check_shape(int64_t N, int64_t K, int64_t G) {
+    if (N <= 0 || K <= 0 || G <= 0) return W4A16_ERR_INVALID_ARG;
+    if (N % 8 || K % 8 || G % 16) return W4A16_ERR_UNSUPPORTED;
+    if (N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    return W4A16_OK;
+}
+
+void fill_scale_plan(Params& p) {
+    const int G = p.G;
+    if (G % 64 == 0) {
+        p.scale_mode = 0;
+        p.scale_rows = 1;
+    } else if (G == 32) {
+        p.scale_mode = 1;
+        p.scale_rows = 2;
+    } else if (G == 16) {
+        p.scale_mode = 2;
+        p.scale_rows = 4;
+    } else {
+        p.scale_mode = 3;
+        p.scale_rows = 64 / G + 2;
+    }
+    if (p.scale_rows > kMaxScaleRows) p.scale_rows = kMaxScaleRows;
+}
+
+struct Plan {
+    int bn;
+    int splits;
+    dim3 grid;
+    int smem;
+    int ctas_per_sm;
+};
+
+int plan_dense(int64_t M, int64_t N, int64_t K, Plan* plan, bool need_device) {
+    const int bn = token_tile_for(M);
+    const int vi = variant_index(bn);
+    int per_sm = kVariants[vi].nominal_per_sm, sms = 148;
+    if (need_device) {
+        DeviceState* st = nullptr;
+        int rc = prepare_device(&st);
+        if (rc) return rc;
+        per_sm = st->ctas_per_sm[vi];
+        sms = sm_count();
+    }
+    const int64_t NT = (N + kTileN - 1) / kTileN;
+    const int64_t MT = (M + bn - 1) / bn;
+    const int64_t KT = (K + kTileK - 1) / kTileK;
+    if (NT > 65535 || MT > 65535) return W4A16_ERR_UNSUPPORTED;
+    int splits = 1;
+    if (MT == 1) {
+        const int64_t slots = static_cast<int64_t>(sms) * per_sm;
+        while (splits < 8 && NT * splits * 2 <= slots && KT >= splits * 4) splits *= 2;
+    }
+    plan->bn = bn;
+    plan->splits = splits;
+    plan->grid = dim3(static_cast<unsigned>(splits), static_cast<unsigned>(NT), static_cast<unsigned>(MT));
+    plan->smem = kVariants[vi].smem;
+    plan->ctas_per_sm = per_sm;
+    return W4A16_OK;
+}
+
+int plan_grouped(int64_t E, int64_t total_rows, int64_t N, int64_t K, Plan* plan, bool need_device) {
+    // Token tile sized for an expert's average row count with headroom, so that
+    // most experts need one tile; each tile's MMA covers only its valid rows
+    // rounded up to 16.
+    const int64_t avg = (total_rows + E - 1) / E;
+    const int bn = token_tile_for(avg + avg / 4);
+    const int vi = variant_index(bn);
+    int per_sm = kVariants[vi].nominal_per_sm;
+    if (need_device) {
+        DeviceState* st = nullptr;
+        int rc = prepare_device(&st);
+        if (rc) return rc;
+        per_sm = st->ctas_per_sm[vi];
+    }
+    const int64_t NT = (N + kTileN - 1) / kTileN;
+    const int64_t slots = total_rows / bn + E;  // >= sum over experts of ceil(rows_e / bn)
+    if (NT > 65535 || slots > 65535) return W4A16_ERR_UNSUPPORTED;
+    (void)K;
+    plan->bn = bn;
+    plan->splits = 1;
+    plan->grid = dim3(1, static_cast<unsigned>(NT), static_cast<unsigned>(slots));
+    plan->smem = kVariants[vi].smem;
+    plan->ctas_per_sm = per_sm;
+    return W4A16_OK;
+}
+
+int make_act_map(CUtensorMap* map, const void* A, int64_t rows, int64_t K, int bn) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return W4A16_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(bn)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(A), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void fill_info(const Plan& plan, w4a16_launch_info* info) {
+    info->token_tile = plan.bn;
+    info->k_splits = plan.splits;
+    info->grid_x = static_cast<int32_t>(plan.grid.x);
+    info->grid_y = static_cast<int32_t>(plan.grid.y);
+    info->grid_z = static_cast<int32_t>(plan.grid.z);
+    info->threads_per_cta = kThreads;
+    info->smem_bytes = plan.smem;
+    info->ctas_per_sm = plan.ctas_per_sm;
+}
+
+}  // namespace
+
+int check_device() {
+    static int cached[64];
+    static bool known[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return W4A16_ERR_UNSUPPORTED;
+    }
+    if (dev < 0 || dev >= 64) return W4A16_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!known[dev]) {
+        int major = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return W4A16_ERR_UNSUPPORTED;
+        }
+        cached[dev] = (major == 10) ? W4A16_OK : W4A16_ERR_UNSUPPORTED;
+        known[dev] = true;
+    }
+    return cached[dev];
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+}  // namespace w4a16
+
+using namespace w4a16;
+
+extern "C" const char* w4a16_status_string(int status) {
+    switch (status) {
+        case W4A16_OK: return "ok";
+        case W4A16_ERR_INVALID_ARG: return "invalid argument";
+        case W4A16_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case W4A16_ERR_UNSUPPORTED: return "unsupported shape or device";
+        case W4A16_ERR_CUDA: return "CUDA runtime error";
+        case W4A16_ERR_TIMEOUT: return "bounded device wait ran out";
+        case W4A16_ERR_BAD_OFFSETS: return "malformed expert offsets";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int w4a16_gemm_launch_info(int64_t M, int64_t N, int64_t K, int64_t G, w4a16_launch_info* info) {
+    if (!info || M <= 0) return W4A16_ERR_INVALID_ARG;
+    int rc = check_shape(N, K, G);
+    if (rc) return rc;
+    if (M >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    const bool dev = check_device() == W4A16_OK;
+    Plan plan;
+    rc = plan_dense(M, N, K, &plan, dev);
+    if (rc) return rc;
+    fill_info(plan, info);
+    return W4A16_OK;
+}
+
+extern "C" int w4a16_grouped_launch_info(int64_t E, int64_t total_rows, int64_t N, int64_t K, int64_t G,
+                                         w4a16_launch_info* info) {
+    if (!info || E <= 0 || E > W4A16_MAX_EXPERTS || total_rows <= 0) return W4A16_ERR_INVALID_ARG;
+    int rc = check_shape(N, K, G);
+    if (rc) return rc;
+    if (total_rows >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    const bool dev = check_device() == W4A16_OK;
+    Plan plan;
+    rc = plan_grouped(E, total_rows, N, K, &plan, dev);
+    if (rc) return rc;
+    fill_info(plan, info);
+    return W4A16_OK;
+}
+
+extern "C" int w4a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt_dev, const w4a16_half* S_dev,
+                          w4a16_half* C_dev, int64_t M, int64_t N, int64_t K, int64_t G, void* stream) {
+    if (!A_dev || !Wt_dev || !S_dev || !C_dev || M < 0) return W4A16_ERR_INVALID_ARG;
+    int rc = check_shape(N, K, G);
+    if (rc) return rc;
+    if (M >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    if (!aligned16(A_dev) || !aligned16(Wt_dev) || !aligned16(S_dev) ||
+        (reinterpret_cast<uintptr_t>(C_dev) & 1u))
+        return W4A16_ERR_MISALIGNED;
+    if (M == 0) return W4A16_OK;
+    rc = check_device();
+    if (rc) return rc;
+    Plan plan;
+    rc = plan_dense(M, N, K, &plan, true);
+    if (rc) return rc;
+
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.wt[0] = Wt_dev;
+    p.sc[0] = reinterpret_cast<const __half*>(S_dev);
+    p.offsets = nullptr;
+    p.C = reinterpret_cast<__half*>(C_dev);
+    p.rows = static_cast<int32_t>(M);
+    p.N = static_cast<int32_t>(N);
+    p.K = static_cast<int32_t>(K);
+    p.G = static_cast<int32_t>(G);
+    p.ngroups = static_cast<int32_t>((K + G - 1) / G);
+    p.KT = static_cast<int32_t>((K + kTileK - 1) / kTileK);
+    p.E = 1;
+    p.splits = plan.splits;
+    p.grouped = 0;
+    fill_scale_plan(p);
+
+    CUtensorMap map;
+    rc = make_act_map(&map, A_dev, M, K, plan.bn);
+    if (rc) return rc;
+    const Variant& v = variant_for(plan.bn);
+    return v.launch(map, p, plan.grid, plan.splits, v.smem, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const* Wt, const w4a16_half* const* S,
+                                  const int32_t* offsets_dev, w4a16_half* C_dev, int64_t E, int64_t total_rows,
+                                  int64_t N, int64_t K, int64_t G, void* stream) {
+    if (!A_dev || !Wt || !S || !offsets_dev || !C_dev || E <= 0 || E > W4A16_MAX_EXPERTS || total_rows < 0)
+        return W4A16_ERR_INVALID_ARG;
+    int rc = check_shape(N, K, G);
+    if (rc) return rc;
+    if (total_rows >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    for (int64_t e = 0; e < E; ++e) {
+        if (!Wt[e] || !S[e]) return W4A16_ERR_INVALID_ARG;
+        if (!aligned16(Wt[e]) || !aligned16(S[e])) return W4A16_ERR_MISALIGNED;
+    }
+    if (!aligned16(A_dev) || (reinterpret_cast<uintptr_t>(C_dev) & 1u) ||
+        (reinterpret_cast<uintptr_t>(offsets_dev) & 3u))
+        return W4A16_ERR_MISALIGNED;
+    if (total_rows == 0) return W4A16_OK;
+    rc = check_device();
+    if (rc) return rc;
+    Plan plan;
+    rc = plan_grouped(E, total_rows, N, K, &plan, true);
+    if (rc) return rc;
+
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    for (int64_t e = 0; e < E; ++e) {
+        p.wt[e] = Wt[e];
+        p.sc[e] = reinterpret_cast<const __half*>(S[e]);
+    }
+    p.offsets = offsets_dev;
+    p.C = reinterpret_cast<__half*>(C_dev);
+    p.rows = static_cast<int32_t>(total_rows);
+    p.N = static_cast<int32_t>(N);
+    p.K = static_cast<int32_t>(K);
+    p.G = static_cast<int32_t>(G);
+    p.ngroups = static_cast<int32_t>((K + G - 1) / G);
+    p.KT = static_cast<int32_t>((K + kTileK - 1) / kTileK);
+    p.E = static_cast<int32_t>(E);
+    p.splits = 1;
+    p.grouped = 1;
+    fill_scale_plan(p);
+
+    CUtensorMap map;
+    rc = make_act_map(&map, A_dev, total_rows, K, plan.bn);
+    if (rc) return rc;
+    const Variant& v = variant_for(plan.bn);
+    return v.launch(map, p, plan.grid, 1, v.smem, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int w4a16_device_status(int clear) {
+    if (check_device() != W4A16_OK) return W4A16_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return W4A16_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return W4A16_ERR_CUDA;
+    if (clear && v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return W4A16_ERR_CUDA;
+    }
+    return v;
+}
