@@ -338,6 +338,7 @@ def run_ours(args):
                      "kernel": "w4a16_gemm_kernel<16,8,2,2> (token tile 16, K split over a cluster)"},
         "e2e": e2e,
         "gpu_launches": world * 2 * K,
+        "launch": {f"M={m}": w4.w4a16_gemm_launch_info(m, N_DIM, K_DIM, G_DIM)[1].as_dict() for m in M_STEP},
         "clocks": clocks,
     }
     if rank == 0:
@@ -464,6 +465,34 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(args):
+    """A few plain launches of one workload family, for ncu (no timing, no rotation)."""
+    import torch
+    from weight_only_int4_wise_b200 import build as wbuild
+    wbuild.build()
+    import weight_only_int4_wise_b200 as w4
+    c = workloads.make(args.profile)
+    dev = torch.device("cuda", 0)
+    if isinstance(c, workloads.DenseCase):
+        _, wt = w4.prepare_weights(torch.from_numpy(c.q).to(dev))
+        A, S = torch.from_numpy(c.A).to(dev), torch.from_numpy(c.S).to(dev)
+        C = torch.empty((c.M, c.N), dtype=torch.float16, device=dev)
+        for _ in range(args.launches):
+            w4.gemm(A, wt, S, c.N, c.G, out=C)
+    else:
+        wts = [w4.prepare_weights(torch.from_numpy(c.q[e]).to(dev))[1] for e in range(c.E)]
+        Ss = [torch.from_numpy(c.S[e]).to(dev) for e in range(c.E)]
+        A, off = torch.from_numpy(c.A).to(dev), torch.from_numpy(c.offsets).to(dev)
+        C = torch.empty((c.total_rows, c.N), dtype=torch.float16, device=dev)
+        for _ in range(args.launches):
+            w4.grouped_gemm(A, wts, Ss, off, c.N, c.G, out=C)
+    torch.cuda.synchronize()
+    status = w4.device_status(clear=True)
+    if status != w4.OK:
+        raise RuntimeError(w4.status_string(status))
+    print(f"profiled {args.profile}: {args.launches} launches")
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -472,10 +501,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config timings")
+    ap.add_argument("--profile", choices=sorted(workloads.CONFIGS), help="only launch this workload (for ncu)")
+    ap.add_argument("--launches", type=int, default=4, help="launches in --profile mode")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -98,9 +98,14 @@ def test_pack_rejects_bad_arguments_on_host(lib):
 
 
 def test_launch_plan_on_host(lib):
-    # Nominal plans (no device here): decode splits K across a cluster; prefill tiles M.
+    # Nominal plans (no device here): decode runs the skinny kernel with K split across a
+    # cluster (8-row token tiles for M <= 8, 16 for M <= 16); prefill tiles M on the tensor-core kernel.
     rc, info = w.w4a16_gemm_launch_info(1, 4096, 4096, 128)
-    assert rc == w.OK and info.token_tile == 16 and info.k_splits > 1 and info.grid_y == 32
+    assert rc == w.OK and info.token_tile == 8 and info.k_splits > 1 and info.grid_y == 32
+    rc, info = w.w4a16_gemm_launch_info(16, 4096, 4096, 128)
+    assert rc == w.OK and info.token_tile == 16 and info.threads_per_cta == 256
+    rc, info = w.w4a16_gemm_launch_info(17, 4096, 4096, 128)
+    assert rc == w.OK and info.token_tile == 32 and info.threads_per_cta == 320
     rc, info = w.w4a16_gemm_launch_info(2048, 4096, 4096, 128)
     assert rc == w.OK and info.token_tile == 256 and info.k_splits == 1 and info.grid_z == 8
     rc, info = w.w4a16_grouped_launch_info(8, 1024, 14336, 4096, 128)

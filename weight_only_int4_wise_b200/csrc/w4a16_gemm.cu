@@ -34,9 +34,11 @@
 
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/w4a16.h"
+#include "dequant.cuh"
 #include "ptx.cuh"
 #include "w4a16_internal.h"
 
@@ -47,12 +49,13 @@ __device__ int g_status;  // latched device-side error (0 = none)
 constexpr int kTileN = 128;                 // weight columns per CTA (MMA M)
 constexpr int kTileK = 64;                  // K per pipeline stage
 constexpr int kRawBytes = 4096;             // int4 codes of one 128 x 64 tile
-constexpr int kW16Bytes = kTileN * kTileK * 2;  // dequantised fp16 tile
+constexpr int kSlotCols = kTileK / 2;       // TMEM columns of one dequantised 128 x 64 fp16 tile
 constexpr int kMaxScaleRows = 4;            // scale rows one stage can touch (G >= 16)
 constexpr int kScaleRowBytes = kTileN * 2;
 constexpr int kDequantWarps = 8;
 constexpr int kThreads = (2 + kDequantWarps) * 32;
-constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per wait
+constexpr int kEarlyStages = 3;            // stages issued before the TMEM allocation sync
+constexpr long long kTimeoutCycles = 4000000000ll;  // about 2 s per wait at the boost clock
 
 struct Params {
     const uint8_t* wt[W4A16_MAX_EXPERTS];   // tiled weights (dense: [0])
@@ -70,37 +73,47 @@ struct Params {
     int32_t grouped;
 };
 
-template <int BN, int LS, int WS>
+// One ring of LS stages. Stage s owns, in shared memory, an activation tile, an
+// int4 tile and its scale rows, and, in tensor memory, a 32-column slot for the
+// dequantised fp16 weights; TMEM also holds the fp32 accumulator (BN columns).
+template <int BN, int LS, int TMEM_COLS>
 struct Layout {
     static constexpr int kActBytes = BN * 128;
     static constexpr int kAct = 0;
-    static constexpr int kW16 = kAct + LS * kActBytes;
-    static constexpr int kRaw = kW16 + WS * kW16Bytes;
+    static constexpr int kRaw = kAct + LS * kActBytes;
     static constexpr int kScale = kRaw + LS * kRawBytes;
     static constexpr int kInfo = kScale + LS * kMaxScaleRows * kScaleRowBytes;  // int2 per stage
     static constexpr int kBar = kInfo + LS * 8;
-    static constexpr int kNumBars = 2 * LS + 2 * WS + 1;
+    static constexpr int kNumBars = 3 * LS + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base, abort flag, tile info
     static constexpr int kTotal = kMisc + 32;
     static constexpr int kAlloc = kTotal + 1024;       // slack for aligning the base to 1024
-    static constexpr int kTmemCols = BN < 32 ? 32 : BN;
-    static constexpr int kRedBytes = BN * kTileN * 4;  // split-K partials, alias the operand rings
-    static_assert(kRedBytes <= kW16 + WS * kW16Bytes, "split-K buffer must fit in the operand rings");
-    static_assert((kActBytes % 1024) == 0 && (kW16 % 1024) == 0, "operand tiles need 1024-byte alignment");
+    static constexpr int kAccCols = BN < 32 ? 32 : BN;
+    static constexpr int kRedBytes = BN * kTileN * 4;  // split-K partials, alias the load ring
+    static_assert(kAccCols + LS * kSlotCols <= TMEM_COLS, "TMEM ring does not fit the allocation");
+    static_assert(TMEM_COLS == 32 || TMEM_COLS == 64 || TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512,
+                  "TMEM allocations are powers of two");
+    static_assert(kRedBytes <= kScale, "split-K buffer must fit in the load ring");
+    static_assert((kActBytes % 1024) == 0, "activation tiles need 1024-byte alignment");
 };
 
 __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
 
 // Bounded wait on an mbarrier phase. Returns false if the CTA is aborting or
-// the wait ran out (which starts the abort).
+// the wait ran out (which starts the abort). The bound is counted in SM clock
+// cycles (clock64 is a cheap, SM-local register; the global timer is far slower
+// to read and would add its latency to every pipeline hand-off).
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
+    long long start = 0;
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
+        if ((it & 15u) == 0) {
             if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kTimeoutNs) {
+            const long long now = clock64();
+            if (start == 0) {
+                start = now;
+            } else if (now - start > kTimeoutCycles) {
                 *abort_flag = 1;
                 latch_status(W4A16_ERR_TIMEOUT);
                 return false;
@@ -112,12 +125,17 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volat
 // Bounded wait that ignores the abort flag: used where in-flight asynchronous
 // work must finish before its resources are released.
 __device__ __forceinline__ bool drain_phase(uint64_t* bar, uint32_t parity) {
-    const uint64_t t0 = global_timer_ns();
+    long long start = 0;
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 63u && global_timer_ns() - t0 > kTimeoutNs) {
-            latch_status(W4A16_ERR_TIMEOUT);
-            return false;
+        if ((it & 15u) == 15u) {
+            const long long now = clock64();
+            if (start == 0) {
+                start = now;
+            } else if (now - start > kTimeoutCycles) {
+                latch_status(W4A16_ERR_TIMEOUT);
+                return false;
+            }
         }
     }
 }
@@ -141,48 +159,18 @@ __device__ __forceinline__ void warp_drain_phase(uint64_t* bar, uint32_t parity)
     if (ok) mbar_try_wait(bar, parity);
 }
 
-__device__ __forceinline__ uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
-__device__ __forceinline__ __half2 bits_h2(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
-
-// Eight int4 codes of one word (nibble i = k_local {0,2,4,6,1,3,5,7}[i]) ->
-// eight fp16 weights q*s in natural k order. Each code c is read as the fp16
-// number 1024 + (c ^ 8) (or 1024 + 16*(c ^ 8) for the high nibble of a byte)
-// by OR-ing it under the exponent of 1024; subtracting the bias then gives the
-// signed code exactly, and one multiply applies the group scale.
-__device__ __forceinline__ uint4 dequant_word(uint32_t x, __half2 s2) {
-    const __half2 bias_lo = bits_h2(0x64086408u);  // 1032, 1032
-    const __half2 sixteenth = bits_h2(0x2C002C00u);  // 1/16, 1/16
-    const __half2 bias_hi = bits_h2(0xD480D480u);  // -72, -72
-    const uint32_t b0 = lop3_and_xor(x, 0x000F000Fu, 0x64086408u);
-    const uint32_t t0 = lop3_and_xor(x, 0x00F000F0u, 0x64806480u);
-    const uint32_t x8 = x >> 8;
-    const uint32_t b1 = lop3_and_xor(x8, 0x000F000Fu, 0x64086408u);
-    const uint32_t t1 = lop3_and_xor(x8, 0x00F000F0u, 0x64806480u);
-    const __half2 q01 = __hsub2(bits_h2(b0), bias_lo);
-    const __half2 q23 = __hfma2(bits_h2(t0), sixteenth, bias_hi);
-    const __half2 q45 = __hsub2(bits_h2(b1), bias_lo);
-    const __half2 q67 = __hfma2(bits_h2(t1), sixteenth, bias_hi);
-    uint4 out;
-    out.x = h2_bits(__hmul2(q01, s2));
-    out.y = h2_bits(__hmul2(q23, s2));
-    out.z = h2_bits(__hmul2(q45, s2));
-    out.w = h2_bits(__hmul2(q67, s2));
-    return out;
-}
-
-template <int BN, int LS, int WS, int MINB>
+template <int BN, int LS, int TMEM_COLS, int MINB>
 __global__ void __launch_bounds__(kThreads, MINB)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ Params p) {
-    using L = Layout<BN, LS, WS>;
+    using L = Layout<BN, LS, TMEM_COLS>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base_addr = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (base_addr & 1023u)) & 1023u);
 
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
-    uint64_t* empty = full + LS;
-    uint64_t* wfull = empty + LS;
-    uint64_t* wempty = wfull + WS;
-    uint64_t* accfull = wempty + WS;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);   // stage's copies landed
+    uint64_t* afull = full + LS;                                     // stage's TMEM weights written
+    uint64_t* done = afull + LS;                                     // stage's MMAs completed
+    uint64_t* accfull = done + LS;                                   // accumulator complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     int* tile_info = reinterpret_cast<int*>(smem + L::kMisc + 8);  // has_tile, expert, m0, rows
@@ -238,78 +226,87 @@ __global__ void __launch_bounds__(kThreads, MINB)
     const int n_mma = min(BN, (rows + 15) & ~15);
     const uint32_t idesc = idesc_f16_f32(128, static_cast<uint32_t>(n_mma));
 
+    // Stage i reads int4 tile kt = kb + i; its scale rows start at g0(i) = floor(kt*64/G),
+    // which the producer tracks incrementally.
+    const uint8_t* wsrc = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes;
+    const __half* ssrc = p.sc[expert] + static_cast<int64_t>(nt) * kTileN;
+    const uint32_t srow_bytes = static_cast<uint32_t>(min(kTileN, p.N - nt * kTileN)) * 2u;
+    int next_k = kb * kTileK;              // first k of the next stage to issue
+    int next_g = next_k / p.G;             // its first scale row
+    int next_i = 0;                        // next stage to issue
+    auto issue_next = [&]() {              // producer thread only
+        const int i = next_i++;
+        const int s = i % LS;
+        while ((next_g + 1) * p.G <= next_k) ++next_g;
+        const int g0 = next_g;
+        const int nrows = min(p.scale_rows, p.ngroups - g0);
+        stage_info[s] = make_int2(g0, nrows);
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kActBytes + kRawBytes) + nrows * srow_bytes);
+        bulk_g2s(smem + L::kRaw + s * kRawBytes, wsrc + static_cast<int64_t>(kb + i) * kRawBytes, kRawBytes, &full[s]);
+        tma_load_2d(smem + L::kAct + s * L::kActBytes, &tmA, next_k, m0, &full[s]);
+        for (int r = 0; r < nrows; ++r)
+            bulk_g2s(smem + L::kScale + (s * kMaxScaleRows + r) * kScaleRowBytes,
+                     ssrc + static_cast<int64_t>(g0 + r) * p.N, srow_bytes, &full[s]);
+        next_k += kTileK;
+    };
+
     if (threadIdx.x == 0) {
         for (int s = 0; s < LS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + kDequantWarps);
-        }
-        for (int w = 0; w < WS; ++w) {
-            mbar_init(&wfull[w], kDequantWarps);
-            mbar_init(&wempty[w], 1);
+            mbar_init(&afull[s], kDequantWarps);
+            mbar_init(&done[s], 1);
         }
         mbar_init(accfull, 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensor_map(&tmA);
+        // Start the first copies before waiting for the TMEM allocation.
+        for (int i = 0; i < min(kEarlyStages, nst); ++i) issue_next();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, L::kTmemCols);
+        tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    const uint32_t tmem_acc = *tmem_slot;
+    const uint32_t tmem_acc = *tmem_slot;                 // accumulator: columns [0, BN)
+    const uint32_t tmem_ring = tmem_acc + L::kAccCols;    // weight slots: kSlotCols columns each
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
+        // A stage's slot is free again once the MMAs that read it completed
+        // (which also means the dequantisation warps finished reading it).
         if (lane == 0) {
-            const uint8_t* wsrc = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes;
-            const __half* ssrc = p.sc[expert] + static_cast<int64_t>(nt) * kTileN;
-            const int ncols = min(kTileN, p.N - nt * kTileN);
-            const uint32_t srow_bytes = static_cast<uint32_t>(ncols) * 2u;
-            int issued = 0;
-            for (int i = 0; i < nst; ++i) {
-                const int s = i % LS;
-                if (i >= LS && !wait_phase(&empty[s], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
+            while (next_i < nst) {
+                const int i = next_i;
+                if (i >= LS && !wait_phase(&done[i % LS], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
                     break;
-                const int kt = kb + i;
-                const int g0 = (kt * kTileK) / p.G;
-                const int nrows = min(p.scale_rows, p.ngroups - g0);
-                stage_info[s] = make_int2(g0, nrows);
-                const uint32_t bytes = static_cast<uint32_t>(L::kActBytes + kRawBytes) + nrows * srow_bytes;
-                mbar_arrive_expect_tx(&full[s], bytes);
-                tma_load_2d(smem + L::kAct + s * L::kActBytes, &tmA, kt * kTileK, m0, &full[s]);
-                bulk_g2s(smem + L::kRaw + s * kRawBytes, wsrc + static_cast<int64_t>(kt) * kRawBytes, kRawBytes,
-                         &full[s]);
-                for (int r = 0; r < nrows; ++r)
-                    bulk_g2s(smem + L::kScale + (s * kMaxScaleRows + r) * kScaleRowBytes,
-                             ssrc + static_cast<int64_t>(g0 + r) * p.N, srow_bytes, &full[s]);
-                issued = i + 1;
+                issue_next();
             }
             // Every issued copy must land before the CTA's shared memory is released.
-            for (int i = max(0, issued - LS); i < issued; ++i)
+            for (int i = max(0, next_i - LS); i < next_i; ++i)
                 drain_phase(&full[i % LS], static_cast<uint32_t>(i / LS) & 1u);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
+            const uint64_t bdesc0 = smem_desc_k_sw128(smem_addr(smem + L::kAct));
             for (int i = 0; i < nst; ++i) {
                 const int s = i % LS;
-                const int w = i % WS;
+                // afull implies the dequantisation warps saw this stage's copies land;
+                // the full-barrier check is then immediate.
+                if (!wait_phase(&afull[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
                 if (!wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
-                if (!wait_phase(&wfull[w], static_cast<uint32_t>(i / WS) & 1u, abort_flag)) break;
                 tc_fence_after_sync();
-                const uint32_t a0 = smem_addr(smem + L::kW16 + w * kW16Bytes);
-                const uint32_t b0 = smem_addr(smem + L::kAct + s * L::kActBytes);
-#pragma unroll
-                for (int kk = 0; kk < kTileK / 16; ++kk) {
-                    mma_f16_ss(tmem_acc, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
-                               (i | kk) != 0 ? 1u : 0u);
-                }
-                mma_commit(&empty[s]);
-                mma_commit(&wempty[w]);
+                const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((s * L::kActBytes) >> 4);
+                const uint32_t a0 = tmem_ring + s * kSlotCols;
+                mma_f16_ts(tmem_acc, a0, bdesc, idesc, i > 0 ? 1u : 0u);
+                mma_f16_ts(tmem_acc, a0 + 8, bdesc + 2, idesc, 1u);
+                mma_f16_ts(tmem_acc, a0 + 16, bdesc + 4, idesc, 1u);
+                mma_f16_ts(tmem_acc, a0 + 24, bdesc + 6, idesc, 1u);
+                mma_commit(&done[s]);
             }
             mma_commit(accfull);  // fires once every MMA issued above has completed
         }
@@ -319,12 +316,12 @@ __global__ void __launch_bounds__(kThreads, MINB)
         const int dw = warp - 2;
         const int h = dw >> 2;            // which 32-deep half of the stage
         const int quad = warp & 3;        // TMEM lane quadrant this warp may access
-        const int j = quad * 32 + lane;   // weight column inside the tile
+        const int j = quad * 32 + lane;   // weight column inside the tile = TMEM lane
         const int n = nt * kTileN + j;
         const bool col_ok = n < p.N;
+        const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
         for (int i = 0; i < nst; ++i) {
             const int s = i % LS;
-            const int w = i % WS;
             if (!warp_wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
             const uint4 raw =
                 *reinterpret_cast<const uint4*>(smem + L::kRaw + s * kRawBytes + h * 2048 + j * 16);
@@ -348,26 +345,29 @@ __global__ void __launch_bounds__(kThreads, MINB)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) sv[q] = srow[min((k0 + 8 * q) / p.G - info.x, last) * kTileN + j];
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-
-            uint4 o0 = dequant_word(raw.x, __half2half2(sv[0]));
-            uint4 o1 = dequant_word(raw.y, __half2half2(sv[1]));
-            uint4 o2 = dequant_word(raw.z, __half2half2(sv[2]));
-            uint4 o3 = dequant_word(raw.w, __half2half2(sv[3]));
-            if (!col_ok) o0 = o1 = o2 = o3 = make_uint4(0, 0, 0, 0);
-
-            if (i >= WS && !warp_wait_phase(&wempty[w], static_cast<uint32_t>((i / WS) - 1) & 1u, abort_flag))
+            uint32_t v[16];
+            {
+                const uint4 o0 = dequant_word(raw.x, __half2half2(sv[0]));
+                const uint4 o1 = dequant_word(raw.y, __half2half2(sv[1]));
+                const uint4 o2 = dequant_word(raw.z, __half2half2(sv[2]));
+                const uint4 o3 = dequant_word(raw.w, __half2half2(sv[3]));
+                v[0] = o0.x; v[1] = o0.y; v[2] = o0.z; v[3] = o0.w;
+                v[4] = o1.x; v[5] = o1.y; v[6] = o1.z; v[7] = o1.w;
+                v[8] = o2.x; v[9] = o2.y; v[10] = o2.z; v[11] = o2.w;
+                v[12] = o3.x; v[13] = o3.y; v[14] = o3.z; v[15] = o3.w;
+            }
+            if (!col_ok) {
+#pragma unroll
+                for (int t = 0; t < 16; ++t) v[t] = 0u;
+            }
+            if (i >= LS && !warp_wait_phase(&done[s], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
                 break;
-            uint8_t* row = smem + L::kW16 + w * kW16Bytes + j * 128;
-            const int sw = j & 7;
-            *reinterpret_cast<uint4*>(row + (((4 * h + 0) ^ sw) << 4)) = o0;
-            *reinterpret_cast<uint4*>(row + (((4 * h + 1) ^ sw) << 4)) = o1;
-            *reinterpret_cast<uint4*>(row + (((4 * h + 2) ^ sw) << 4)) = o2;
-            *reinterpret_cast<uint4*>(row + (((4 * h + 3) ^ sw) << 4)) = o3;
-            fence_proxy_async_smem();
+            tc_fence_after_sync();
+            tmem_st_32x32b_x16(tmem_ring + tlane + s * kSlotCols + h * 16, v);
+            tmem_st_wait();
+            tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&wfull[w]);
+            if (lane == 0) mbar_arrive(&afull[s]);
         }
 
         // -------------------------------------------------- epilogue
@@ -377,7 +377,6 @@ __global__ void __launch_bounds__(kThreads, MINB)
         tc_fence_after_sync();
         const int aborted = __shfl_sync(0xffffffffu, *abort_flag, 0);
         const bool have_acc = !aborted && nst > 0;
-        const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
         if (p.splits == 1) {
             if (have_acc) {
                 __half* cbase = p.C + static_cast<int64_t>(m0) * p.N + n;
@@ -415,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem_acc, L::kTmemCols);
+        tmem_dealloc(tmem_acc, TMEM_COLS);
     }
 
     if (p.splits > 1) {
@@ -432,8 +431,13 @@ __global__ void __launch_bounds__(kThreads, MINB)
             const int tok = o / cw;
             const int nn = nt * kTileN + col;
             if (nn < p.N && !aborted) {
+                float part[8];
+#pragma unroll
+                for (int src = 0; src < 8; ++src)
+                    part[src] = src < S ? ld_dsmem_f32(&red[tok * kTileN + col], static_cast<uint32_t>(src)) : 0.f;
                 float acc = 0.f;
-                for (int src = 0; src < S; ++src) acc += ld_dsmem_f32(&red[tok * kTileN + col], static_cast<uint32_t>(src));
+#pragma unroll
+                for (int src = 0; src < 8; ++src) acc += part[src];  // rank order
                 p.C[static_cast<int64_t>(m0 + tok) * p.N + nn] = __float2half_rn(acc);
             }
         }
@@ -466,12 +470,13 @@ EncodeTiledFn encode_fn() {
 struct Variant {
     int bn;
     int nominal_per_sm;  // the residency the variant is sized for (used when no device is present)
+    int tmem_cols;       // TMEM columns each resident CTA allocates
     int smem;
     const void* fn;
     int (*launch)(const CUtensorMap&, const Params&, dim3, int, int, cudaStream_t);
 };
 
-template <int BN, int LS, int WS, int MINB>
+template <int BN, int LS, int TC, int MINB>
 int launch_variant(const CUtensorMap& map, const Params& p, dim3 grid, int cluster_x, int smem, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -488,20 +493,22 @@ int launch_variant(const CUtensorMap& map, const Params& p, dim3 grid, int clust
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    cudaError_t e = cudaLaunchKernelEx(&cfg, w4a16_gemm_kernel<BN, LS, WS, MINB>, map, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, w4a16_gemm_kernel<BN, LS, TC, MINB>, map, p);
     return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
-template <int BN, int LS, int WS, int MINB>
+template <int BN, int LS, int TC, int MINB>
 Variant make_variant() {
-    return Variant{BN, MINB, Layout<BN, LS, WS>::kAlloc, reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, WS, MINB>),
-                   &launch_variant<BN, LS, WS, MINB>};
+    return Variant{BN, MINB, TC, Layout<BN, LS, TC>::kAlloc,
+                   reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB>),
+                   &launch_variant<BN, LS, TC, MINB>};
 }
 
 // Token tiles and their pipeline depths: small tiles keep two CTAs per SM.
+// <token tile, ring stages, TMEM columns, CTAs per SM>
 const Variant kVariants[] = {
-    make_variant<16, 8, 2, 2>(),  make_variant<32, 8, 2, 2>(),  make_variant<64, 5, 2, 2>(),
-    make_variant<128, 5, 2, 1>(), make_variant<256, 4, 2, 1>(),
+    make_variant<16, 7, 256, 2>(), make_variant<32, 7, 256, 2>(), make_variant<64, 6, 256, 2>(),
+    make_variant<128, 4, 256, 2>(), make_variant<256, 5, 512, 1>(),
 };
 
 const Variant& variant_for(int bn) {
@@ -525,14 +532,25 @@ int prepare_device(DeviceState** out) {
     if (!st.ready) {
         for (int i = 0; i < 5; ++i) {
             const Variant& v = kVariants[i];
-            if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess)
+            if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess ||
+                cudaFuncSetAttribute(v.fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared) != cudaSuccess)
                 return W4A16_ERR_CUDA;
-            int n = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, v.fn, kThreads, v.smem) != cudaSuccess || n < 1)
-                return W4A16_ERR_CUDA;
-            // Every resident CTA holds TMEM columns; never ask for more than the SM has.
-            const int cols = v.bn < 32 ? 32 : v.bn;
-            if (n * cols > 512) n = 512 / cols;
+            // Residency from the SM's limits (shared memory with its per-block
+            // reservation, registers per warp, threads, TMEM columns).
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, v.fn) != cudaSuccess) return W4A16_ERR_CUDA;
+            int smem_sm = 0, resv = 0, regs_sm = 0, threads_sm = 0;
+            cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+            cudaDeviceGetAttribute(&resv, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+            cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+            cudaDeviceGetAttribute(&threads_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
+            const int per_warp_regs = ((fa.numRegs * 32 + 255) / 256) * 256;
+            int n = smem_sm / (v.smem + static_cast<int>(fa.sharedSizeBytes) + resv);
+            n = std::min(n, regs_sm / (per_warp_regs * (kThreads / 32)));
+            n = std::min(n, threads_sm / kThreads);
+            n = std::min(n, 512 / v.tmem_cols);  // every resident CTA holds its TMEM columns
+            if (n < 1) return W4A16_ERR_UNSUPPORTED;
             st.ctas_per_sm[i] = n;
         }
         st.ready = true;
@@ -723,6 +741,18 @@ extern "C" int w4a16_gemm_launch_info(int64_t M, int64_t N, int64_t K, int64_t G
     if (rc) return rc;
     if (M >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
     const bool dev = check_device() == W4A16_OK;
+    SkinnyPlan sk;
+    if (skinny_plan(M, N, K, G, &sk) == W4A16_OK) {
+        info->token_tile = 8 * sk.mt;
+        info->k_splits = sk.splits;
+        info->grid_x = sk.grid_x;
+        info->grid_y = sk.grid_y;
+        info->grid_z = 1;
+        info->threads_per_cta = 256;
+        info->smem_bytes = sk.smem;
+        info->ctas_per_sm = (228 * 1024) / (sk.smem + 1024) < 2 ? (228 * 1024) / (sk.smem + 1024) : 2;
+        return W4A16_OK;
+    }
     Plan plan;
     rc = plan_dense(M, N, K, &plan, dev);
     if (rc) return rc;
@@ -756,6 +786,9 @@ extern "C" int w4a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt_dev, const 
     if (M == 0) return W4A16_OK;
     rc = check_device();
     if (rc) return rc;
+    SkinnyPlan sk;
+    if (skinny_plan(M, N, K, G, &sk) == W4A16_OK)
+        return skinny_launch(sk, A_dev, Wt_dev, S_dev, C_dev, M, N, K, G, static_cast<cudaStream_t>(stream));
     Plan plan;
     rc = plan_dense(M, N, K, &plan, true);
     if (rc) return rc;

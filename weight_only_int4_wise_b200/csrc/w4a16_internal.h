@@ -3,6 +3,8 @@
 
 #include <cuda_runtime.h>
 
+#include <cstdint>
+
 #include "../../include/w4a16.h"
 
 namespace w4a16 {
@@ -13,5 +15,25 @@ int check_device();
 
 // Streaming multiprocessors of the current device (0 if unknown).
 int sm_count();
+
+// Decode-sized products (M <= kSkinnyMaxM) run on the skinny kernel.
+constexpr int kSkinnyMaxM = 16;
+
+struct SkinnyPlan {
+    int mt;             // token tiles of 8 rows (1 or 2)
+    int splits;         // CTAs along K in one cluster
+    int grid_x, grid_y;
+    int act_stride;     // staged activation row, in halves
+    int scale_rows;     // staged scale rows
+    int smem;           // dynamic shared memory per CTA
+    uint32_t g_magic;   // multiply-shift constant for floor(k / G)
+    int post_scale;     // 1 when every 128-deep K block lies in one scale group
+};
+
+// W4A16_OK and a plan, or W4A16_ERR_UNSUPPORTED if the shape needs the general kernel.
+int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan);
+
+int skinny_launch(const SkinnyPlan& plan, const void* A, const uint8_t* Wt, const void* S, void* C, int64_t M,
+                  int64_t N, int64_t K, int64_t G, cudaStream_t stream);
 
 }  // namespace w4a16
