@@ -230,6 +230,11 @@ def run_ours(args):
         if rc:
             raise RuntimeError(w4.status_string(rc))
 
+    # Weights and scales are prepared once, before any timing, and never written
+    # again: declare them static so each GEMM may stream them before the previous
+    # kernel on the stream finishes (activations and outputs still wait for it).
+    torch.cuda.synchronize()
+    w4.w4a16_set_static_weights(True)
     # warm the library's per-device setup outside any capture
     launch(1, 0)
     launch(16, 1)
@@ -330,7 +335,8 @@ def run_ours(args):
         "config": {"workload": WORKLOAD, "M": list(M_STEP), "K": K_DIM, "N": N_DIM, "G": G_DIM,
                    "l2": f"inputs larger than L2: {R} rotating copies of weights+scales+activations "
                          f"({R * copy_bytes / 2 ** 20:.0f} MiB vs {l2 / 2 ** 20:.0f} MiB L2)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "static_weights": True, "launch": "CUDA graphs, programmatic dependent launch"},
         "tflops": round(tflops, 3),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic_from_profile(),

@@ -116,6 +116,19 @@ int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const* Wt, const 
                        const int32_t* offsets_dev, w4a16_half* C_dev, int64_t E, int64_t total_rows,
                        int64_t N, int64_t K, int64_t G, void* stream);
 
+/* Declares (enable != 0) or withdraws (enable == 0) the promise that no
+ * kernel on the calling streams writes the tiled weights or the scales passed
+ * to w4a16_gemm right before that call, i.e. the weights are static (prepared
+ * once, as at model load time). Every GEMM kernel is launched with
+ * programmatic dependent launch, so it may start while the previous kernel on
+ * its stream is still running; it always waits for that kernel before reading
+ * activations or writing the output. With static weights declared, the dense
+ * kernels also start streaming Wt and S before that wait, which hides the
+ * launch and memory-latency ramp between back-to-back GEMMs. Process-wide;
+ * off by default. Returns the previous setting. Has no counterpart on the
+ * plugin pages. */
+int w4a16_set_static_weights(int enable);
+
 /* How w4a16_gemm / w4a16_grouped_gemm will launch for a shape (no work is
  * enqueued): the token tile (MMA N extent), the K split, the grid and the
  * CTAs per SM. Errors as for the GEMM's host validation. */

@@ -226,3 +226,45 @@ def test_full_size_grouped_sampled(o):
         ref = o.gemm_sample(c.A[r0:r1], pins.python_pack(c.q[e]), c.S[e], c.K, c.G, rows, cols)
         ok, err, rel = within_tolerance(got[r0 + rows, cols], ref)
         assert ok, f"grouped expert {e}: max abs err {err}, max rel err {rel}"
+
+
+def test_static_weights_mode(o):
+    # Weights prepared (and synchronised) well before the GEMMs: with static weights
+    # declared the kernels may stream them before the previous kernel finishes.
+    cases = [workloads.make("decode_m16"), workloads.dense(8, 4096, 2048, 128, 51), workloads.dense(40, 1024, 640, 64, 52)]
+    prepared = [(c, device_weights(c.q)[1], dev(c.A), dev(c.S)) for c in cases]
+    torch.cuda.synchronize()
+    previous = w.w4a16_set_static_weights(True)
+    try:
+        outs = [w.gemm(A, wt, S, c.N, c.G) for c, wt, A, S in prepared for _ in range(2)]
+        torch.cuda.synchronize()
+    finally:
+        w.w4a16_set_static_weights(previous)
+    for idx, (c, _, _, _) in enumerate(prepared):
+        ref = o.gemm(c.A, pins.python_pack(c.q), c.S, c.K, c.G)
+        for got in outs[2 * idx:2 * idx + 2]:
+            ok, err, rel = within_tolerance(got.cpu().numpy(), ref)
+            assert ok, f"static weights, case {idx}: max abs err {err}"
+
+
+def test_repack_then_gemm_back_to_back(o):
+    # The GEMM right after the repack kernel that produced its weights, on one stream.
+    for c in (workloads.dense(8, 4096, 14336, 128, 53), workloads.dense(16, 14336, 1024, 128, 54)):
+        _, wt = device_weights(c.q)
+        got = w.gemm(dev(c.A), wt, dev(c.S), c.N, c.G).cpu().numpy()
+        ref = o.gemm(c.A, pins.python_pack(c.q), c.S, c.K, c.G)
+        ok, err, rel = within_tolerance(got, ref)
+        assert ok, f"repack then gemm: max abs err {err}"
+
+
+def test_stage_refill_is_race_free(o):
+    # K ranges longer than the skinny kernel's ring (so stages are refilled while
+    # other warps still compute) must give the same bits on every run.
+    for c in (workloads.dense(8, 4096, 14336, 128, 55), workloads.dense(16, 14336, 4096, 64, 56)):
+        _, wt = device_weights(c.q)
+        A, S = dev(c.A), dev(c.S)
+        runs = [w.gemm(A, wt, S, c.N, c.G).cpu().numpy() for _ in range(4)]
+        for r in runs[1:]:
+            assert np.array_equal(r.view(np.uint16), runs[0].view(np.uint16))
+        ok, err, _ = within_tolerance(runs[0], o.gemm(c.A, pins.python_pack(c.q), c.S, c.K, c.G))
+        assert ok, f"max abs err {err}"

@@ -28,7 +28,7 @@ MAX_EXPERTS = 64
 EXPORTED = [
     "w4a16_status_string", "w4a16_pack", "w4a16_unpack", "w4a16_tiled_bytes", "w4a16_repack",
     "w4a16_gemm", "w4a16_grouped_gemm", "w4a16_gemm_launch_info", "w4a16_grouped_launch_info",
-    "w4a16_device_status",
+    "w4a16_device_status", "w4a16_set_static_weights",
 ]
 
 
@@ -79,6 +79,8 @@ def load() -> ctypes.CDLL:
         lib.w4a16_grouped_launch_info.restype = ctypes.c_int
         lib.w4a16_device_status.argtypes = [ctypes.c_int]
         lib.w4a16_device_status.restype = ctypes.c_int
+        lib.w4a16_set_static_weights.argtypes = [ctypes.c_int]
+        lib.w4a16_set_static_weights.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -154,6 +156,11 @@ def w4a16_grouped_launch_info(E: int, total_rows: int, N: int, K: int, G: int):
 
 def w4a16_device_status(clear: bool = True) -> int:
     return int(load().w4a16_device_status(1 if clear else 0))
+
+
+def w4a16_set_static_weights(enable: bool) -> int:
+    """Declare weights and scales static (see include/w4a16.h); returns the previous setting."""
+    return int(load().w4a16_set_static_weights(1 if enable else 0))
 
 
 # ------------------------------------------------------------- torch helpers

@@ -35,6 +35,7 @@
 #include <cstdint>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/w4a16.h"
@@ -71,6 +72,7 @@ struct Params {
     int32_t scale_rows; // scale rows fetched per stage
     int32_t scale_mode; // 0: G % 64 == 0, 1: G == 32, 2: G == 16, 3: other
     int32_t grouped;
+    int32_t prefetch;   // weights/scales may be read before the previous kernel finishes
 };
 
 // One ring of LS stages. Stage s owns, in shared memory, an activation tile, an
@@ -184,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     if (threadIdx.x == 0) {
         int has = 1, expert = 0, m0 = 0, rows = 0;
         if (p.grouped) {
+            grid_dependency_wait();  // the offsets may come from the previous kernel
             const int32_t* off = p.offsets;
             bool ok = off[0] == 0 && off[p.E] == p.rows;
             for (int e = 0; e < p.E && ok; ++e) ok = off[e + 1] >= off[e];
@@ -234,7 +237,9 @@ __global__ void __launch_bounds__(kThreads, MINB)
     int next_k = kb * kTileK;              // first k of the next stage to issue
     int next_g = next_k / p.G;             // its first scale row
     int next_i = 0;                        // next stage to issue
-    auto issue_next = [&]() {              // producer thread only
+    // Weights and scale rows of the next stage (read-only, safe before the
+    // previous kernel finishes); the activation tile follows with issue_act.
+    auto issue_wts = [&]() {               // producer thread only
         const int i = next_i++;
         const int s = i % LS;
         while ((next_g + 1) * p.G <= next_k) ++next_g;
@@ -243,13 +248,17 @@ __global__ void __launch_bounds__(kThreads, MINB)
         stage_info[s] = make_int2(g0, nrows);
         mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kActBytes + kRawBytes) + nrows * srow_bytes);
         bulk_g2s(smem + L::kRaw + s * kRawBytes, wsrc + static_cast<int64_t>(kb + i) * kRawBytes, kRawBytes, &full[s]);
-        tma_load_2d(smem + L::kAct + s * L::kActBytes, &tmA, next_k, m0, &full[s]);
         for (int r = 0; r < nrows; ++r)
             bulk_g2s(smem + L::kScale + (s * kMaxScaleRows + r) * kScaleRowBytes,
                      ssrc + static_cast<int64_t>(g0 + r) * p.N, srow_bytes, &full[s]);
         next_k += kTileK;
     };
+    auto issue_act = [&](int i) {
+        const int s = i % LS;
+        tma_load_2d(smem + L::kAct + s * L::kActBytes, &tmA, (kb + i) * kTileK, m0, &full[s]);
+    };
 
+    const int early = p.prefetch ? min(kEarlyStages, nst) : 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < LS; ++s) {
             mbar_init(&full[s], 1);
@@ -260,8 +269,10 @@ __global__ void __launch_bounds__(kThreads, MINB)
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensor_map(&tmA);
-        // Start the first copies before waiting for the TMEM allocation.
-        for (int i = 0; i < min(kEarlyStages, nst); ++i) issue_next();
+        // With static weights (set by the caller), start the first weight copies
+        // before waiting for the TMEM allocation and for the previous kernel.
+        for (int i = 0; i < early; ++i) issue_wts();
+        grid_launch_dependents();
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -278,11 +289,14 @@ __global__ void __launch_bounds__(kThreads, MINB)
         // A stage's slot is free again once the MMAs that read it completed
         // (which also means the dequantisation warps finished reading it).
         if (lane == 0) {
+            grid_dependency_wait();  // anything but static weights may be written by the previous kernel
+            for (int i = 0; i < early; ++i) issue_act(i);
             while (next_i < nst) {
                 const int i = next_i;
                 if (i >= LS && !wait_phase(&done[i % LS], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
                     break;
-                issue_next();
+                issue_wts();
+                issue_act(i);
             }
             // Every issued copy must land before the CTA's shared memory is released.
             for (int i = max(0, next_i - LS); i < next_i; ++i)
@@ -375,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
         // either way no MMA may still run when TMEM is released.
         warp_drain_phase(accfull, 0);
         tc_fence_after_sync();
+        grid_dependency_wait();  // the output may still be read by the previous kernel
         const int aborted = __shfl_sync(0xffffffffu, *abort_flag, 0);
         const bool have_acc = !aborted && nst > 0;
         if (p.splits == 1) {
@@ -483,16 +498,20 @@ int launch_variant(const CUtensorMap& map, const Params& p, dim3 grid, int clust
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    cfg.numAttrs = 0;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
     if (cluster_x > 1) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = static_cast<unsigned>(cluster_x);
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
     }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
     cudaError_t e = cudaLaunchKernelEx(&cfg, w4a16_gemm_kernel<BN, LS, TC, MINB>, map, p);
     return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
@@ -711,6 +730,12 @@ int check_device() {
     return cached[dev];
 }
 
+namespace {
+std::atomic<int> g_static_weights{0};
+}
+
+bool static_weights_enabled() { return g_static_weights.load(std::memory_order_relaxed) != 0; }
+
 int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -733,6 +758,11 @@ extern "C" const char* w4a16_status_string(int status) {
         case W4A16_ERR_BAD_OFFSETS: return "malformed expert offsets";
         default: return "unknown status";
     }
+}
+
+extern "C" int w4a16_set_static_weights(int enable) {
+    const int previous = g_static_weights.exchange(enable ? 1 : 0);
+    return previous;
 }
 
 extern "C" int w4a16_gemm_launch_info(int64_t M, int64_t N, int64_t K, int64_t G, w4a16_launch_info* info) {
@@ -808,6 +838,7 @@ extern "C" int w4a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt_dev, const 
     p.E = 1;
     p.splits = plan.splits;
     p.grouped = 0;
+    p.prefetch = static_weights_enabled() ? 1 : 0;
     fill_scale_plan(p);
 
     CUtensorMap map;
@@ -856,6 +887,7 @@ extern "C" int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const*
     p.E = static_cast<int32_t>(E);
     p.splits = 1;
     p.grouped = 1;
+    p.prefetch = 0;  // expert weights are read only after the offsets, which follow the wait
     fill_scale_plan(p);
 
     CUtensorMap map;
@@ -874,5 +906,7 @@ extern "C" int w4a16_device_status(int clear) {
         const int zero = 0;
         if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return W4A16_ERR_CUDA;
     }
-    return v;
+    const int vs = skinny_device_status(clear != 0);
+    if (vs < 0) return W4A16_ERR_CUDA;
+    return v != 0 ? v : vs;
 }

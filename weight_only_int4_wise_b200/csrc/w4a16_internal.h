@@ -16,12 +16,16 @@ int check_device();
 // Streaming multiprocessors of the current device (0 if unknown).
 int sm_count();
 
+// Whether the caller declared weights and scales static (w4a16_set_static_weights).
+bool static_weights_enabled();
+
 // Decode-sized products (M <= kSkinnyMaxM) run on the skinny kernel.
 constexpr int kSkinnyMaxM = 16;
 
 struct SkinnyPlan {
     int mt;             // token tiles of 8 rows (1 or 2)
     int splits;         // CTAs along K in one cluster
+    int depth;          // 128-deep K blocks in flight per thread (4 or 8)
     int grid_x, grid_y;
     int act_stride;     // staged activation row, in halves
     int scale_rows;     // staged scale rows
@@ -32,6 +36,9 @@ struct SkinnyPlan {
 
 // W4A16_OK and a plan, or W4A16_ERR_UNSUPPORTED if the shape needs the general kernel.
 int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan);
+
+// The skinny kernel's latched device status (0 = none, -1 if it could not be read).
+int skinny_device_status(bool clear);
 
 int skinny_launch(const SkinnyPlan& plan, const void* A, const uint8_t* Wt, const void* S, void* C, int64_t M,
                   int64_t N, int64_t K, int64_t G, cudaStream_t stream);
