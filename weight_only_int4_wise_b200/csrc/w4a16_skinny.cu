@@ -3,13 +3,13 @@
 // The operation is the Int4GroupwiseGemmPluginV2 page's (class description:
 // activations, int4 weights, scales [ceil(K/G),N], fp16 output). At M <= 16 the
 // product is bound by streaming the int4 weights from HBM (K*N/2 bytes):
-//   - a producer warp moves each 128-deep K block of a 128-column weight tile
-//     (8 KB, contiguous in the tiled layout) with one bulk copy into a ring of
-//     kDepth shared-memory stages, completing on that stage's mbarrier;
-//   - eight compute warps (16 output columns each) read their fragments from a
-//     stage, release it at once, and decode them straight into the A operand
-//     of a warp-level m16n8k16 MMA (weights as the 16-row operand, tokens as
-//     the 8-column operand: one or two token tiles);
+//   - each thread streams its own two 16-byte int4 chunks per 128-deep K block
+//     with cp.async into a private ring of kDepth blocks (per-thread copies
+//     keep more requests in flight per SM than one bulk engine does, and no
+//     thread ever reads another thread's slot, so stages need no barrier);
+//   - it decodes them straight into the A operand of a warp-level m16n8k16
+//     MMA (weights as the 16-row operand, 16 output columns per warp; tokens
+//     as the 8-column operand: one or two token tiles);
 //   - scale rows ride on the first stage; activations are staged after the
 //     previous kernel in the stream has finished (programmatic dependent
 //     launch lets the weight copies start before that);
@@ -37,30 +37,15 @@ namespace w4a16 {
 
 namespace {
 
-constexpr int kSkWarps = 8;                       // compute warps: 8 x 16 columns = one 128-column tile
-constexpr int kSkThreads = (kSkWarps + 1) * 32;   // plus one producer warp
+constexpr int kSkWarps = 8;                       // 8 warps x 16 columns = one 128-column weight tile
+constexpr int kSkThreads = kSkWarps * 32;
 constexpr int kBlockK = 128;
-constexpr int kBlockBytes = 8192;                 // int4 codes of a 128-column x 128-deep block
-constexpr long long kSkTimeoutCycles = 4000000000ll;
+constexpr int kSlotBytes = 32;                    // per thread and block: two 16-byte chunks
 
-__device__ int g_skinny_status;  // latched device-side error of this kernel (0 = none)
-
-// Bounded wait on an mbarrier phase (SM-clock bound). False on timeout, which is latched.
-__device__ __forceinline__ bool sk_wait(uint64_t* bar, uint32_t parity) {
-    long long start = 0;
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 15u) == 15u) {
-            const long long now = clock64();
-            if (start == 0) {
-                start = now;
-            } else if (now - start > kSkTimeoutCycles) {
-                atomicCAS(&g_skinny_status, 0, W4A16_ERR_TIMEOUT);
-                return false;
-            }
-        }
-    }
-}
+// No wait in this kernel can fail to end (cp.async groups and cluster barriers
+// only), so its status word stays 0; it is kept so the device-status query has
+// one word per kernel family.
+__device__ int g_skinny_status;
 
 struct SkinnyParams {
     const uint8_t* wt;      // tiled weights
@@ -92,52 +77,59 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
     const int S = p.splits;
     const int cwm = (128 + S - 1) / S;              // widest output-column slice of one cluster rank
 
-    uint8_t* ring = sm;                                                   // [kDepth][8 KB]
-    __half* act = reinterpret_cast<__half*>(ring + kDepth * kBlockBytes); // [MP][act_stride]
+    __half* act = reinterpret_cast<__half*>(sm);                          // [MP][act_stride]
     __half* scl = act + MP * p.act_stride;                                // [scale_rows][128]
-    float* red = reinterpret_cast<float*>(scl + p.scale_rows * 128);      // [S][MP][cwm] split-K partials
-    uint64_t* full = reinterpret_cast<uint64_t*>(red + (S > 1 ? S * MP * cwm : 0));
-    uint64_t* empty = full + kDepth;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kDepth);
+    uint8_t* ring = reinterpret_cast<uint8_t*>(scl + p.scale_rows * 128); // [kDepth][2][threads][16 B]
+    float* red = reinterpret_cast<float*>(ring + kDepth * kSkThreads * kSlotBytes);  // [S][MP][cwm] partials
 
     const int g_lo = kr0 / p.G;
     const int g_hi = min(p.ngroups - 1, (kr0 + krange - 1) / p.G);
     const int nrows = g_hi - g_lo + 1;
-    const uint32_t srow_bytes = static_cast<uint32_t>(min(128, p.N - nt * 128)) * 2u;
-    const uint8_t* wsrc = p.wt + (static_cast<int64_t>(nt) * p.KT + 2 * b0) * 4096;
-    // Block i holds tiles 2(b0+i) and 2(b0+i)+1; the second is missing at an odd end of K.
-    auto block_bytes = [&](int i) { return 2 * (b0 + i) + 1 < p.KT ? kBlockBytes : kBlockBytes / 2; };
-    auto issue = [&](int i) {  // producer lane only
-        const int s = i % kDepth;
-        uint32_t bytes = static_cast<uint32_t>(block_bytes(i));
-        if (i == 0) bytes += nrows * srow_bytes;
-        mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_g2s(ring + s * kBlockBytes, wsrc + static_cast<int64_t>(i) * kBlockBytes, block_bytes(i), &full[s]);
-        if (i == 0)
-            for (int r = 0; r < nrows; ++r)
-                bulk_g2s(scl + r * 128, p.sc + static_cast<int64_t>(g_lo + r) * p.N + nt * 128, srow_bytes, &full[0]);
+    const int ja = warp * 16 + g;  // this thread's columns: ja and ja + 8
+
+    // This thread's chunk t of columns ja and ja + 8 in block i: tile 2(b0+i) + t/2,
+    // half t%2. A missing second tile at an odd end of K reads as zeros.
+    const uint8_t* wsrc = p.wt + (static_cast<int64_t>(nt) * p.KT + 2 * b0 + (t >> 1)) * 4096 + (t & 1) * 2048 + ja * 16;
+    const int kt_last_ok = p.KT - 1 - (t >> 1);
+    uint8_t* myslot = ring + threadIdx.x * 16;  // chunk of column ja; column ja + 8's is kSkThreads * 16 further
+    auto issue_block = [&](int i) {
+        if (i < nb) {
+            const bool ok = 2 * (b0 + i) <= kt_last_ok;
+            const uint8_t* src = wsrc + static_cast<int64_t>(i) * 8192;
+            uint8_t* dst = myslot + (i % kDepth) * kSkThreads * kSlotBytes;
+            cp_async16(dst, ok ? src : p.wt, ok ? 16u : 0u);
+            cp_async16(dst + kSkThreads * 16, ok ? src + 128 : p.wt, ok ? 16u : 0u);
+        }
+        cp_async_commit();  // one group per block, empty past the end, so the counts stay uniform
+    };
+    auto issue_scales = [&]() {
+        const int ncols = min(128, p.N - nt * 128);
+        for (int idx = threadIdx.x; idx < nrows * 16; idx += kSkThreads) {
+            const int r = idx >> 4, c = idx & 15;
+            const bool ok = c * 8 < ncols;
+            cp_async16(scl + r * 128 + c * 8,
+                       ok ? p.sc + static_cast<int64_t>(g_lo + r) * p.N + nt * 128 + c * 8 : p.sc, ok ? 16u : 0u);
+        }
+        cp_async_commit();  // the oldest group: complete by the time block 0 is
     };
 
-    // ---- with static weights (set by the caller) the weight and scale copies
-    // start before the previous kernel in the stream has finished
-    const bool producer = warp == kSkWarps;
-    if (producer && lane == 0) {
-        for (int s = 0; s < kDepth; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kSkWarps);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-        if (p.prefetch)
-            for (int i = 0; i < min(kDepth, nb); ++i) issue(i);
+    // ---- with static weights (declared by the caller) the scale and weight
+    // copies start before the previous kernel in the stream has finished
+    if (p.prefetch) {
+        issue_scales();
+#pragma unroll
+        for (int i = 0; i < kDepth; ++i) issue_block(i);
     }
 
     // ---- everything else may come from the previous kernel: wait for it, then
     // stage the activations with plain loads (zero past M and K)
     grid_launch_dependents();
     grid_dependency_wait();
-    if (producer && lane == 0 && !p.prefetch)
-        for (int i = 0; i < min(kDepth, nb); ++i) issue(i);
+    if (!p.prefetch) {
+        issue_scales();
+#pragma unroll
+        for (int i = 0; i < kDepth; ++i) issue_block(i);
+    }
     {
         const int cpr = krange / 8;  // 16-byte chunks per activation row
         for (int idx = threadIdx.x; idx < MP * cpr; idx += kSkThreads) {
@@ -148,143 +140,92 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
             *reinterpret_cast<uint4*>(act + r * p.act_stride + c * 8) = v;
         }
     }
-    __syncthreads();  // staged activations and the barrier initialisation are visible
+    __syncthreads();  // staged activations are visible; scales are waited for with block 0
 
     float acc[MT][4];
 #pragma unroll
     for (int j = 0; j < MT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-    const int ja = (warp < kSkWarps ? warp : 0) * 16 + g;  // this thread's columns: ja and ja + 8
+    uint32_t arow[MT];
+#pragma unroll
+    for (int j = 0; j < MT; ++j) arow[j] = smem_addr(act + (8 * j + g) * p.act_stride + 32 * t);
+    const uint32_t slot0 = smem_addr(myslot);
 
-    if (producer) {
-        // ------------------------------------------------ refill freed stages
-        if (lane == 0) {
-            int issued = min(kDepth, nb);
-            for (int i = kDepth; i < nb && !*abort_flag; ++i) {
-                const int s = i % kDepth;
-                if (!sk_wait(&empty[s], static_cast<uint32_t>((i / kDepth) - 1) & 1u)) {
-                    *abort_flag = 1;
-                    break;
-                }
-                fence_proxy_async_smem();  // the warps' reads of the stage precede the copy's writes
-                issue(i);
-                issued = i + 1;
-            }
-            // every issued copy lands before the CTA's shared memory is released
-            for (int i = max(0, issued - kDepth); i < issued; ++i)
-                if (!sk_wait(&full[i % kDepth], static_cast<uint32_t>(i / kDepth) & 1u)) *abort_flag = 1;
-        }
-        __syncwarp();
-    } else {
-        // ------------------------------------------------ compute
-        uint32_t arow[MT];
+    for (int i = 0; i < nb; ++i) {
+        cp_async_wait<kDepth - 1>();  // block i (and the scales) are in this thread's slot
+        if (i == 0) __syncthreads();  // the scale rows were copied by all threads
+        const uint32_t slot = slot0 + (i % kDepth) * kSkThreads * kSlotBytes;
+        const uint4 wa = lds128(slot);
+        const uint4 wb = lds128(slot + kSkThreads * 16);
+        const uint32_t kb2 = static_cast<uint32_t>(i * kBlockK * 2);  // block offset in the staged range, bytes
+        const uint32_t wa_w[4] = {wa.x, wa.y, wa.z, wa.w};
+        const uint32_t wb_w[4] = {wb.x, wb.y, wb.z, wb.w};
+        if (p.post_scale) {
+            // One group covers the whole block: one MMA chain over the exact codes,
+            // started from a zero accumulator, then one scaled add per element.
+            float part[MT][4];
 #pragma unroll
-        for (int j = 0; j < MT; ++j) arow[j] = smem_addr(act + (8 * j + g) * p.act_stride + 32 * t);
-        // chunk t of column ja: tile t/2 of the block, half t%2
-        const uint32_t frag0 = smem_addr(ring) + (t >> 1) * 4096 + (t & 1) * 2048 + ja * 16;
-        for (int i = 0; i < nb; ++i) {
-            const int s = i % kDepth;
-            int ok = 1;
-            if (lane == 0) ok = sk_wait(&full[s], static_cast<uint32_t>(i / kDepth) & 1u) ? 1 : 0;
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) {
-                *abort_flag = 1;
-                break;
-            }
-            mbar_try_wait(&full[s], static_cast<uint32_t>(i / kDepth) & 1u);  // completed: acquire for every lane
-            uint4 wa = make_uint4(0u, 0u, 0u, 0u), wb = wa;
-            if (!(t >> 1) || block_bytes(i) == kBlockBytes) {
-                wa = lds128(frag0 + s * kBlockBytes);
-                wb = lds128(frag0 + s * kBlockBytes + 128);
-            }
-            const uint32_t kb2 = static_cast<uint32_t>(i * kBlockK * 2);  // block offset in the staged range, bytes
-            const uint32_t wa_w[4] = {wa.x, wa.y, wa.z, wa.w};
-            const uint32_t wb_w[4] = {wb.x, wb.y, wb.z, wb.w};
-            if (p.post_scale) {
-                // One group covers the whole block: one MMA chain over the exact codes,
-                // started from a zero accumulator, then one scaled add per element.
-                uint4 qa_all[4], qb_all[4];
+            for (int w = 0; w < 4; ++w) {
+                const uint4 qa = decode_word(wa_w[w]);
+                const uint4 qb = decode_word(wb_w[w]);
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    qa_all[w] = decode_word(wa_w[w]);
-                    qb_all[w] = decode_word(wb_w[w]);
-                }
-                // The stage's bytes are all decoded (so both loads have completed):
-                // it may be refilled while this warp runs its MMAs.
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-                float part[MT][4];
+                for (int u = 0; u < 2; ++u) {
+                    const uint32_t afr[4] = {u ? qa.z : qa.x, u ? qb.z : qb.x, u ? qa.w : qa.y, u ? qb.w : qb.y};
+                    const int st = 2 * w + u;
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const uint4 qa = qa_all[w];
-                    const uint4 qb = qb_all[w];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const uint32_t afr[4] = {u ? qa.z : qa.x, u ? qb.z : qb.x, u ? qa.w : qa.y, u ? qb.w : qb.y};
-                        const int st = 2 * w + u;
-#pragma unroll
-                        for (int j = 0; j < MT; ++j) {
-                            const uint2 bfr = lds64(arow[j] + kb2 + 8 * st);
-                            if (st == 0)
-                                mma_m16n8k16_zc(part[j], afr, bfr.x, bfr.y);
-                            else
-                                mma_m16n8k16(part[j], afr, bfr.x, bfr.y);
-                        }
+                    for (int j = 0; j < MT; ++j) {
+                        const uint2 bfr = lds64(arow[j] + kb2 + 8 * st);
+                        if (st == 0)
+                            mma_m16n8k16_zc(part[j], afr, bfr.x, bfr.y);
+                        else
+                            mma_m16n8k16(part[j], afr, bfr.x, bfr.y);
                     }
                 }
-                const int gr = (kr0 + i * kBlockK) / p.G - g_lo;
-                const float sa = __half2float(scl[gr * 128 + ja]);
-                const float sb = __half2float(scl[gr * 128 + ja + 8]);
+            }
+            const int gr = (kr0 + i * kBlockK) / p.G - g_lo;
+            const float sa = __half2float(scl[gr * 128 + ja]);
+            const float sb = __half2float(scl[gr * 128 + ja + 8]);
 #pragma unroll
-                for (int j = 0; j < MT; ++j) {
-                    acc[j][0] = fmaf(part[j][0], sa, acc[j][0]);
-                    acc[j][1] = fmaf(part[j][1], sa, acc[j][1]);
-                    acc[j][2] = fmaf(part[j][2], sb, acc[j][2]);
-                    acc[j][3] = fmaf(part[j][3], sb, acc[j][3]);
-                }
-            } else {
-                // Groups finer than the block: scale each decoded word (rounded to fp16).
-                uint4 qa_all[4], qb_all[4];
+            for (int j = 0; j < MT; ++j) {
+                acc[j][0] = fmaf(part[j][0], sa, acc[j][0]);
+                acc[j][1] = fmaf(part[j][1], sa, acc[j][1]);
+                acc[j][2] = fmaf(part[j][2], sb, acc[j][2]);
+                acc[j][3] = fmaf(part[j][3], sb, acc[j][3]);
+            }
+        } else {
+            // Groups finer than the block: scale each decoded word (rounded to fp16).
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const uint32_t kk = static_cast<uint32_t>(kr0 + i * kBlockK + 32 * t + 8 * w);
-                    const int gr =
-                        min(static_cast<int>((static_cast<uint64_t>(kk) * p.g_magic) >> 32), p.ngroups - 1) - g_lo;
-                    qa_all[w] = dequant_word(wa_w[w], __half2half2(scl[gr * 128 + ja]));
-                    qb_all[w] = dequant_word(wb_w[w], __half2half2(scl[gr * 128 + ja + 8]));
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
+            for (int w = 0; w < 4; ++w) {
+                const uint32_t kk = static_cast<uint32_t>(kr0 + i * kBlockK + 32 * t + 8 * w);
+                const int gr =
+                    min(static_cast<int>((static_cast<uint64_t>(kk) * p.g_magic) >> 32), p.ngroups - 1) - g_lo;
+                const uint4 qa = dequant_word(wa_w[w], __half2half2(scl[gr * 128 + ja]));
+                const uint4 qb = dequant_word(wb_w[w], __half2half2(scl[gr * 128 + ja + 8]));
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const uint4 qa = qa_all[w];
-                    const uint4 qb = qb_all[w];
+                for (int u = 0; u < 2; ++u) {
+                    const uint32_t afr[4] = {u ? qa.z : qa.x, u ? qb.z : qb.x, u ? qa.w : qa.y, u ? qb.w : qb.y};
+                    const int st = 2 * w + u;
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const uint32_t afr[4] = {u ? qa.z : qa.x, u ? qb.z : qb.x, u ? qa.w : qa.y, u ? qb.w : qb.y};
-                        const int st = 2 * w + u;
-#pragma unroll
-                        for (int j = 0; j < MT; ++j) {
-                            const uint2 bfr = lds64(arow[j] + kb2 + 8 * st);
-                            mma_m16n8k16(acc[j], afr, bfr.x, bfr.y);
-                        }
+                    for (int j = 0; j < MT; ++j) {
+                        const uint2 bfr = lds64(arow[j] + kb2 + 8 * st);
+                        mma_m16n8k16(acc[j], afr, bfr.x, bfr.y);
                     }
                 }
             }
         }
+        issue_block(i + kDepth);  // this thread's slot for block i is consumed (values decoded above)
     }
+    cp_async_wait<0>();
 
     const int na = nt * 128 + ja;
     if (S == 1) {
-        if (!producer) {
 #pragma unroll
-            for (int j = 0; j < MT; ++j) {
-                const int m0 = 8 * j + 2 * t;
+        for (int j = 0; j < MT; ++j) {
+            const int m0 = 8 * j + 2 * t;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int m = m0 + (e & 1);
-                    const int n = na + ((e >> 1) << 3);
-                    if (m < p.M && n < p.N) p.C[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(acc[j][e]);
-                }
+            for (int e = 0; e < 4; ++e) {
+                const int m = m0 + (e & 1);
+                const int n = na + ((e >> 1) << 3);
+                if (m < p.M && n < p.N) p.C[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(acc[j][e]);
             }
         }
         return;
@@ -295,18 +236,16 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
     // [ceil(q*128/S), ceil((q+1)*128/S))), one cluster barrier publishes them,
     // and each owner sums its S slices in rank order.
     const int rank = static_cast<int>(cluster_ctarank());
-    if (!producer) {
 #pragma unroll
-        for (int j = 0; j < MT; ++j) {
-            const int m0 = 8 * j + 2 * t;
+    for (int j = 0; j < MT; ++j) {
+        const int m0 = 8 * j + 2 * t;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int m = m0 + (e & 1);
-                const int col = ja + ((e >> 1) << 3);
-                const int q = (col * S) >> 7;          // owner of this column
-                const int cq = (q * 128 + S - 1) / S;  // owner's first column
-                if (m < p.M) st_dsmem_f32(&red[(rank * MP + m) * cwm + (col - cq)], static_cast<uint32_t>(q), acc[j][e]);
-            }
+        for (int e = 0; e < 4; ++e) {
+            const int m = m0 + (e & 1);
+            const int col = ja + ((e >> 1) << 3);
+            const int q = (col * S) >> 7;          // owner of this column
+            const int cq = (q * 128 + S - 1) / S;  // owner's first column
+            if (m < p.M) st_dsmem_f32(&red[(rank * MP + m) * cwm + (col - cq)], static_cast<uint32_t>(q), acc[j][e]);
         }
     }
     cluster_sync_all();
@@ -323,9 +262,9 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
 }
 
 int smem_bytes(int mt, int depth, int splits, int act_stride, int scale_rows) {
-    const int ring = depth * kBlockBytes;
+    const int ring = depth * kSkThreads * kSlotBytes;
     const int red = splits > 1 ? splits * 8 * mt * ((128 + splits - 1) / splits) * 4 : 0;
-    return ring + 8 * mt * act_stride * 2 + scale_rows * 256 + red + 2 * depth * 8 + 16;
+    return 8 * mt * act_stride * 2 + scale_rows * 256 + ring + red;
 }
 
 }  // namespace
@@ -338,8 +277,9 @@ int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan) {
     const int mt = M <= 8 ? 1 : 2;
     int sms = sm_count();
     if (sms <= 0) sms = 148;
-    // Enough CTAs for about two per SM, never more than the cluster limit or the K blocks.
-    int64_t splits = (2 * sms + NT - 1) / NT;
+    // Up to two CTAs per SM in a single wave (a second wave of clusters would
+    // double the time), never more than the cluster limit or the K blocks.
+    int64_t splits = (2 * sms) / NT;
     if (splits > 8) splits = 8;
     if (splits > KB) splits = KB;
     if (splits < 1) splits = 1;
