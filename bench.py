@@ -144,6 +144,34 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest of one float per rank (every rank gets it); the identity without a process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, seconds_max: float) -> float:
+    """Whole-job rate: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_rank / seconds_max
+
+
+SKINNY_SOURCES = ("w4a16_skinny.cu", "dequant.cuh", "ptx.cuh")
+
+
+def skinny_source_digest() -> str:
+    """sha256 over the sources that make up the skinny kernel, in a fixed order."""
+    h = hashlib.sha256()
+    for name in SKINNY_SOURCES:
+        with open(os.path.join(ROOT, "weight_only_int4_wise_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def traffic_from_profile():
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the current kernel source."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
@@ -151,9 +179,7 @@ def traffic_from_profile():
         return None
     with open(path) as f:
         d = json.load(f)
-    src = os.path.join(ROOT, "weight_only_int4_wise_b200", "csrc", "w4a16_gemm.cu")
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    if d.get("kernel_source_sha256") != digest:
+    if d.get("kernel_source_sha256") != skinny_source_digest():
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -276,13 +302,10 @@ def run_ours(args):
         dist.barrier()
     ms = e0.elapsed_time(e1)
     clocks = sampler.stop() if rank == 0 else None
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dev)
     sec = ms_max / 1e3
-    value = world * K * step_bytes() / sec / 1e9
-    tflops = world * K * step_flops() / sec / 1e12
+    value = job_throughput(K * step_bytes(), world, sec) / 1e9
+    tflops = job_throughput(K * step_flops(), world, sec) / 1e12
 
     status = w4.device_status(clear=True)
     if status != w4.OK:
@@ -317,11 +340,8 @@ def run_ours(args):
         e2e_step(i)
     f1.record()
     f1.synchronize()
-    te = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_sec = float(te.item()) / 1e3
-    e2e = {"value": world * K_e2e * step_bytes() / e2e_sec / 1e9, "unit": "GB/s",
+    e2e_sec = max_over_ranks(f0.elapsed_time(f1), dev) / 1e3
+    e2e = {"value": job_throughput(K_e2e * step_bytes(), world, e2e_sec) / 1e9, "unit": "GB/s",
            "h2d_bytes_per_step": sum(m * K_DIM * 2 for m in M_STEP),
            "d2h_bytes_per_step": sum(m * N_DIM * 2 for m in M_STEP), "steps": K_e2e}
 
@@ -341,7 +361,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic_from_profile(),
                      "peak_source": f"{peaks['source']} (copy bandwidth)",
-                     "kernel": "w4a16_gemm_kernel<16,8,2,2> (token tile 16, K split over a cluster)"},
+                     "kernel": "w4a16_skinny_kernel (M <= 16: 8- or 16-row token tiles, K split over a cluster)"},
         "e2e": e2e,
         "gpu_launches": world * 2 * K,
         "launch": {f"M={m}": w4.w4a16_gemm_launch_info(m, N_DIM, K_DIM, G_DIM)[1].as_dict() for m in M_STEP},
