@@ -12,16 +12,17 @@
 // on the 5th-generation tensor core: each CTA owns 128 weight columns (the MMA
 // M extent, one TMEM lane per column) and a tile of BN activation rows (the
 // MMA N extent, 16..256), so that small token counts cost no padding of the
-// weight side. Warp roles inside a CTA (320 threads):
+// weight side. Warp roles inside a CTA (320 or 576 threads):
 //   warp 0      producer: per 64-deep K stage, one TMA tile load of the
 //               activations (128-byte swizzle, zero fill past M and K), one
 //               4096-byte bulk copy of the tiled int4 weights and the scale rows.
 //   warp 1      TMEM allocation and the single MMA-issuing thread
 //               (tcgen05.mma kind::f16, fp32 accumulator in TMEM).
-//   warps 2..9  dequantisation: each thread turns 32 int4 codes of one column
-//               into fp16 (magic-exponent decode, times the group scale) and
-//               stores them into the K-major swizzled A-operand tile; then the
-//               epilogue (tcgen05.ld -> fp16 -> global).
+//   warps 2..   dequantisation, in one or two groups of 8 warps (group g takes
+//               stages g, g + groups, ...): each thread turns 32 int4 codes of
+//               one column into fp16 (magic-exponent decode, times the group
+//               scale) and stores them into the stage's tensor-memory slot;
+//               then the epilogue (tcgen05.ld -> fp16 -> global).
 // Small-M shapes split K across up to 8 CTAs of one thread-block cluster; the
 // fp32 partial tiles are summed in rank order through distributed shared
 // memory (deterministic, no global workspace).
@@ -53,8 +54,10 @@ constexpr int kRawBytes = 4096;             // int4 codes of one 128 x 64 tile
 constexpr int kSlotCols = kTileK / 2;       // TMEM columns of one dequantised 128 x 64 fp16 tile
 constexpr int kMaxScaleRows = 4;            // scale rows one stage can touch (G >= 16)
 constexpr int kScaleRowBytes = kTileN * 2;
-constexpr int kDequantWarps = 8;
-constexpr int kThreads = (2 + kDequantWarps) * 32;
+constexpr int kDequantWarps = 8;           // one group: 4 TMEM lane quadrants x 2 halves of a stage
+// Threads of a CTA with DQ dequantisation groups (each group takes every
+// DQ-th stage, so DQ groups keep DQ stages in flight).
+__host__ __device__ constexpr int threads_for(int dq) { return (2 + kDequantWarps * dq) * 32; }
 constexpr int kEarlyStages = 3;            // stages issued before the TMEM allocation sync
 constexpr long long kTimeoutCycles = 4000000000ll;  // about 2 s per wait at the boost clock
 
@@ -86,7 +89,7 @@ struct Layout {
     static constexpr int kScale = kRaw + LS * kRawBytes;
     static constexpr int kInfo = kScale + LS * kMaxScaleRows * kScaleRowBytes;  // int2 per stage
     static constexpr int kBar = kInfo + LS * 8;
-    static constexpr int kNumBars = 3 * LS + 1;
+    static constexpr int kNumBars = 4 * LS + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base, abort flag, tile info
     static constexpr int kTotal = kMisc + 32;
     static constexpr int kAlloc = kTotal + 1024;       // slack for aligning the base to 1024
@@ -161,8 +164,8 @@ __device__ __forceinline__ void warp_drain_phase(uint64_t* bar, uint32_t parity)
     if (ok) mbar_try_wait(bar, parity);
 }
 
-template <int BN, int LS, int TMEM_COLS, int MINB>
-__global__ void __launch_bounds__(kThreads, MINB)
+template <int BN, int LS, int TMEM_COLS, int MINB, int DQ>
+__global__ void __launch_bounds__(threads_for(DQ), MINB)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ Params p) {
     using L = Layout<BN, LS, TMEM_COLS>;
     extern __shared__ uint8_t smem_raw[];
@@ -170,7 +173,8 @@ __global__ void __launch_bounds__(kThreads, MINB)
     uint8_t* smem = smem_raw + ((1024u - (base_addr & 1023u)) & 1023u);
 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);   // stage's copies landed
-    uint64_t* afull = full + LS;                                     // stage's TMEM weights written
+    uint64_t* wfull = full + LS;                                     // stage's int4 tile and scale rows landed
+    uint64_t* afull = wfull + LS;                                    // stage's TMEM weights written
     uint64_t* done = afull + LS;                                     // stage's MMAs completed
     uint64_t* accfull = done + LS;                                   // accumulator complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -246,15 +250,16 @@ __global__ void __launch_bounds__(kThreads, MINB)
         const int g0 = next_g;
         const int nrows = min(p.scale_rows, p.ngroups - g0);
         stage_info[s] = make_int2(g0, nrows);
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kActBytes + kRawBytes) + nrows * srow_bytes);
-        bulk_g2s(smem + L::kRaw + s * kRawBytes, wsrc + static_cast<int64_t>(kb + i) * kRawBytes, kRawBytes, &full[s]);
+        mbar_arrive_expect_tx(&wfull[s], static_cast<uint32_t>(kRawBytes) + nrows * srow_bytes);
+        bulk_g2s(smem + L::kRaw + s * kRawBytes, wsrc + static_cast<int64_t>(kb + i) * kRawBytes, kRawBytes, &wfull[s]);
         for (int r = 0; r < nrows; ++r)
             bulk_g2s(smem + L::kScale + (s * kMaxScaleRows + r) * kScaleRowBytes,
-                     ssrc + static_cast<int64_t>(g0 + r) * p.N, srow_bytes, &full[s]);
+                     ssrc + static_cast<int64_t>(g0 + r) * p.N, srow_bytes, &wfull[s]);
         next_k += kTileK;
     };
     auto issue_act = [&](int i) {
         const int s = i % LS;
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kActBytes));
         tma_load_2d(smem + L::kAct + s * L::kActBytes, &tmA, (kb + i) * kTileK, m0, &full[s]);
     };
 
@@ -262,6 +267,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     if (threadIdx.x == 0) {
         for (int s = 0; s < LS; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&wfull[s], 1);
             mbar_init(&afull[s], kDequantWarps);
             mbar_init(&done[s], 1);
         }
@@ -299,8 +305,10 @@ __global__ void __launch_bounds__(kThreads, MINB)
                 issue_act(i);
             }
             // Every issued copy must land before the CTA's shared memory is released.
-            for (int i = max(0, next_i - LS); i < next_i; ++i)
+            for (int i = max(0, next_i - LS); i < next_i; ++i) {
+                drain_phase(&wfull[i % LS], static_cast<uint32_t>(i / LS) & 1u);
                 drain_phase(&full[i % LS], static_cast<uint32_t>(i / LS) & 1u);
+            }
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -309,8 +317,8 @@ __global__ void __launch_bounds__(kThreads, MINB)
             const uint64_t bdesc0 = smem_desc_k_sw128(smem_addr(smem + L::kAct));
             for (int i = 0; i < nst; ++i) {
                 const int s = i % LS;
-                // afull implies the dequantisation warps saw this stage's copies land;
-                // the full-barrier check is then immediate.
+                // The stage's dequantised weights (afull), then its activation tile (full):
+                // the dequantisation warps only wait for the small int4 and scale copies.
                 if (!wait_phase(&afull[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
                 if (!wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
                 tc_fence_after_sync();
@@ -328,15 +336,16 @@ __global__ void __launch_bounds__(kThreads, MINB)
     } else {
         // ------------------------------------------------------ dequant + epilogue
         const int dw = warp - 2;
-        const int h = dw >> 2;            // which 32-deep half of the stage
+        const int grp = dw >> 3;          // dequantisation group: stages grp, grp + DQ, ...
+        const int h = (dw >> 2) & 1;      // which 32-deep half of the stage
         const int quad = warp & 3;        // TMEM lane quadrant this warp may access
         const int j = quad * 32 + lane;   // weight column inside the tile = TMEM lane
         const int n = nt * kTileN + j;
         const bool col_ok = n < p.N;
         const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
-        for (int i = 0; i < nst; ++i) {
+        for (int i = grp; i < nst; i += DQ) {
             const int s = i % LS;
-            if (!warp_wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
+            if (!warp_wait_phase(&wfull[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
             const uint4 raw =
                 *reinterpret_cast<const uint4*>(smem + L::kRaw + s * kRawBytes + h * 2048 + j * 16);
             const int2 info = stage_info[s];
@@ -395,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
         if (p.splits == 1) {
             if (have_acc) {
                 __half* cbase = p.C + static_cast<int64_t>(m0) * p.N + n;
-                for (int c = h; c < n_mma / 16; c += 2) {
+                for (int c = h + 2 * grp; c < n_mma / 16; c += 2 * DQ) {
                     uint32_t v[16];
                     tmem_ld_32x32b_x16(tmem_acc + tlane + c * 16, v);
                     tmem_ld_wait();
@@ -410,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
             }
         } else {
             float* red = reinterpret_cast<float*>(smem + L::kAct);
-            for (int c = h; c < BN / 16; c += 2) {
+            for (int c = h + 2 * grp; c < BN / 16; c += 2 * DQ) {
                 uint32_t v[16];
                 if (have_acc && c * 16 < n_mma) {
                     tmem_ld_32x32b_x16(tmem_acc + tlane + c * 16, v);
@@ -441,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
         const int rank = static_cast<int>(cluster_ctarank());
         const float* red = reinterpret_cast<const float*>(smem + L::kAct);
         const bool aborted = *abort_flag != 0;
-        for (int o = threadIdx.x; o < cw * rows; o += kThreads) {
+        for (int o = threadIdx.x; o < cw * rows; o += static_cast<int>(blockDim.x)) {
             const int col = rank * cw + (o % cw);
             const int tok = o / cw;
             const int nn = nt * kTileN + col;
@@ -484,6 +493,7 @@ EncodeTiledFn encode_fn() {
 
 struct Variant {
     int bn;
+    int threads;
     int nominal_per_sm;  // the residency the variant is sized for (used when no device is present)
     int tmem_cols;       // TMEM columns each resident CTA allocates
     int smem;
@@ -491,11 +501,11 @@ struct Variant {
     int (*launch)(const CUtensorMap&, const Params&, dim3, int, int, cudaStream_t);
 };
 
-template <int BN, int LS, int TC, int MINB>
+template <int BN, int LS, int TC, int MINB, int DQ>
 int launch_variant(const CUtensorMap& map, const Params& p, dim3 grid, int cluster_x, int smem, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(threads_for(DQ), 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -512,22 +522,24 @@ int launch_variant(const CUtensorMap& map, const Params& p, dim3 grid, int clust
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, w4a16_gemm_kernel<BN, LS, TC, MINB>, map, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, w4a16_gemm_kernel<BN, LS, TC, MINB, DQ>, map, p);
     return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
-template <int BN, int LS, int TC, int MINB>
+template <int BN, int LS, int TC, int MINB, int DQ>
 Variant make_variant() {
-    return Variant{BN, MINB, TC, Layout<BN, LS, TC>::kAlloc,
-                   reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB>),
-                   &launch_variant<BN, LS, TC, MINB>};
+    return Variant{BN, threads_for(DQ), MINB, TC, Layout<BN, LS, TC>::kAlloc,
+                   reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB, DQ>),
+                   &launch_variant<BN, LS, TC, MINB, DQ>};
 }
 
-// Token tiles and their pipeline depths: small tiles keep two CTAs per SM.
-// <token tile, ring stages, TMEM columns, CTAs per SM>
+// Token tiles and their pipeline depths: small tiles keep two CTAs per SM; the
+// 256-row tile (one CTA per SM, MMAs of N = 256) runs two dequantisation
+// groups so that decoding two stages at once keeps pace with the tensor core.
+// <token tile, ring stages, TMEM columns, CTAs per SM, dequantisation groups>
 const Variant kVariants[] = {
-    make_variant<16, 7, 256, 2>(), make_variant<32, 7, 256, 2>(), make_variant<64, 6, 256, 2>(),
-    make_variant<128, 4, 256, 2>(), make_variant<256, 5, 512, 1>(),
+    make_variant<16, 7, 256, 2, 1>(), make_variant<32, 7, 256, 2, 1>(), make_variant<64, 6, 256, 2, 1>(),
+    make_variant<128, 4, 256, 2, 1>(), make_variant<256, 5, 512, 1, 2>(),
 };
 
 const Variant& variant_for(int bn) {
@@ -566,8 +578,8 @@ int prepare_device(DeviceState** out) {
             cudaDeviceGetAttribute(&threads_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
             const int per_warp_regs = ((fa.numRegs * 32 + 255) / 256) * 256;
             int n = smem_sm / (v.smem + static_cast<int>(fa.sharedSizeBytes) + resv);
-            n = std::min(n, regs_sm / (per_warp_regs * (kThreads / 32)));
-            n = std::min(n, threads_sm / kThreads);
+            n = std::min(n, regs_sm / (per_warp_regs * (v.threads / 32)));
+            n = std::min(n, threads_sm / v.threads);
             n = std::min(n, 512 / v.tmem_cols);  // every resident CTA holds its TMEM columns
             if (n < 1) return W4A16_ERR_UNSUPPORTED;
             st.ctas_per_sm[i] = n;
@@ -700,7 +712,7 @@ void fill_info(const Plan& plan, w4a16_launch_info* info) {
     info->grid_x = static_cast<int32_t>(plan.grid.x);
     info->grid_y = static_cast<int32_t>(plan.grid.y);
     info->grid_z = static_cast<int32_t>(plan.grid.z);
-    info->threads_per_cta = kThreads;
+    info->threads_per_cta = variant_for(plan.bn).threads;
     info->smem_bytes = plan.smem;
     info->ctas_per_sm = plan.ctas_per_sm;
 }
