@@ -14,15 +14,16 @@
 // MMA N extent, 16..256), so that small token counts cost no padding of the
 // weight side. Warp roles inside a CTA (320 or 576 threads):
 //   warp 0      producer: per 64-deep K stage, one TMA tile load of the
-//               activations (128-byte swizzle, zero fill past M and K), one
-//               4096-byte bulk copy of the tiled int4 weights and the scale rows.
+//               activations (128-byte swizzle, zero fill past M and K).
 //   warp 1      TMEM allocation and the single MMA-issuing thread
 //               (tcgen05.mma kind::f16, fp32 accumulator in TMEM).
 //   warps 2..   dequantisation, in one or two groups of 8 warps (group g takes
-//               stages g, g + groups, ...): each thread turns 32 int4 codes of
-//               one column into fp16 (magic-exponent decode, times the group
-//               scale) and stores them into the stage's tensor-memory slot;
-//               then the epilogue (tcgen05.ld -> fp16 -> global).
+//               stages g, g + groups, ...): each thread loads 32 int4 codes of
+//               one column (16 bytes of the tiled layout) and their scales
+//               straight into registers two of its stages ahead, turns them
+//               into fp16 (magic-exponent decode, times the group scale) and
+//               stores them into the stage's tensor-memory slot; then the
+//               epilogue (tcgen05.ld -> fp16 -> global).
 // Small-M shapes split K across up to 8 CTAs of one thread-block cluster; the
 // fp32 partial tiles are summed in rank order through distributed shared
 // memory (deterministic, no global workspace).
@@ -52,13 +53,10 @@ constexpr int kTileN = 128;                 // weight columns per CTA (MMA M)
 constexpr int kTileK = 64;                  // K per pipeline stage
 constexpr int kRawBytes = 4096;             // int4 codes of one 128 x 64 tile
 constexpr int kSlotCols = kTileK / 2;       // TMEM columns of one dequantised 128 x 64 fp16 tile
-constexpr int kMaxScaleRows = 4;            // scale rows one stage can touch (G >= 16)
-constexpr int kScaleRowBytes = kTileN * 2;
 constexpr int kDequantWarps = 8;           // one group: 4 TMEM lane quadrants x 2 halves of a stage
 // Threads of a CTA with DQ dequantisation groups (each group takes every
 // DQ-th stage, so DQ groups keep DQ stages in flight).
 __host__ __device__ constexpr int threads_for(int dq) { return (2 + kDequantWarps * dq) * 32; }
-constexpr int kEarlyStages = 3;            // stages issued before the TMEM allocation sync
 constexpr long long kTimeoutCycles = 4000000000ll;  // about 2 s per wait at the boost clock
 
 struct Params {
@@ -72,24 +70,21 @@ struct Params {
     int32_t KT;         // ceil(K/64)
     int32_t E;          // grouped: number of experts; dense: 1
     int32_t splits;     // CTAs along K (cluster size along x)
-    int32_t scale_rows; // scale rows fetched per stage
-    int32_t scale_mode; // 0: G % 64 == 0, 1: G == 32, 2: G == 16, 3: other
     int32_t grouped;
     int32_t prefetch;   // weights/scales may be read before the previous kernel finishes
 };
 
-// One ring of LS stages. Stage s owns, in shared memory, an activation tile, an
-// int4 tile and its scale rows, and, in tensor memory, a 32-column slot for the
-// dequantised fp16 weights; TMEM also holds the fp32 accumulator (BN columns).
+// One ring of LS stages. Stage s owns, in shared memory, an activation tile
+// and, in tensor memory, a 32-column slot for the dequantised fp16 weights;
+// TMEM also holds the fp32 accumulator (BN columns). The int4 codes and the
+// scales go straight from global memory into the dequantising threads'
+// registers, a few stages ahead, so the copy engine only moves activations.
 template <int BN, int LS, int TMEM_COLS>
 struct Layout {
     static constexpr int kActBytes = BN * 128;
     static constexpr int kAct = 0;
-    static constexpr int kRaw = kAct + LS * kActBytes;
-    static constexpr int kScale = kRaw + LS * kRawBytes;
-    static constexpr int kInfo = kScale + LS * kMaxScaleRows * kScaleRowBytes;  // int2 per stage
-    static constexpr int kBar = kInfo + LS * 8;
-    static constexpr int kNumBars = 4 * LS + 1;
+    static constexpr int kBar = kAct + LS * kActBytes;
+    static constexpr int kNumBars = 3 * LS + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base, abort flag, tile info
     static constexpr int kTotal = kMisc + 32;
     static constexpr int kAlloc = kTotal + 1024;       // slack for aligning the base to 1024
@@ -98,7 +93,7 @@ struct Layout {
     static_assert(kAccCols + LS * kSlotCols <= TMEM_COLS, "TMEM ring does not fit the allocation");
     static_assert(TMEM_COLS == 32 || TMEM_COLS == 64 || TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512,
                   "TMEM allocations are powers of two");
-    static_assert(kRedBytes <= kScale, "split-K buffer must fit in the load ring");
+    static_assert(kRedBytes <= kBar, "split-K buffer must fit in the activation ring");
     static_assert((kActBytes % 1024) == 0, "activation tiles need 1024-byte alignment");
 };
 
@@ -173,14 +168,12 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
     uint8_t* smem = smem_raw + ((1024u - (base_addr & 1023u)) & 1023u);
 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);   // stage's copies landed
-    uint64_t* wfull = full + LS;                                     // stage's int4 tile and scale rows landed
-    uint64_t* afull = wfull + LS;                                    // stage's TMEM weights written
+    uint64_t* afull = full + LS;                                     // stage's TMEM weights written
     uint64_t* done = afull + LS;                                     // stage's MMAs completed
     uint64_t* accfull = done + LS;                                   // accumulator complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     int* tile_info = reinterpret_cast<int*>(smem + L::kMisc + 8);  // has_tile, expert, m0, rows
-    int2* stage_info = reinterpret_cast<int2*>(smem + L::kInfo);    // {first scale row, rows valid}
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -233,41 +226,15 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
     const int n_mma = min(BN, (rows + 15) & ~15);
     const uint32_t idesc = idesc_f16_f32(128, static_cast<uint32_t>(n_mma));
 
-    // Stage i reads int4 tile kt = kb + i; its scale rows start at g0(i) = floor(kt*64/G),
-    // which the producer tracks incrementally.
-    const uint8_t* wsrc = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes;
-    const __half* ssrc = p.sc[expert] + static_cast<int64_t>(nt) * kTileN;
-    const uint32_t srow_bytes = static_cast<uint32_t>(min(kTileN, p.N - nt * kTileN)) * 2u;
-    int next_k = kb * kTileK;              // first k of the next stage to issue
-    int next_g = next_k / p.G;             // its first scale row
-    int next_i = 0;                        // next stage to issue
-    // Weights and scale rows of the next stage (read-only, safe before the
-    // previous kernel finishes); the activation tile follows with issue_act.
-    auto issue_wts = [&]() {               // producer thread only
-        const int i = next_i++;
-        const int s = i % LS;
-        while ((next_g + 1) * p.G <= next_k) ++next_g;
-        const int g0 = next_g;
-        const int nrows = min(p.scale_rows, p.ngroups - g0);
-        stage_info[s] = make_int2(g0, nrows);
-        mbar_arrive_expect_tx(&wfull[s], static_cast<uint32_t>(kRawBytes) + nrows * srow_bytes);
-        bulk_g2s(smem + L::kRaw + s * kRawBytes, wsrc + static_cast<int64_t>(kb + i) * kRawBytes, kRawBytes, &wfull[s]);
-        for (int r = 0; r < nrows; ++r)
-            bulk_g2s(smem + L::kScale + (s * kMaxScaleRows + r) * kScaleRowBytes,
-                     ssrc + static_cast<int64_t>(g0 + r) * p.N, srow_bytes, &wfull[s]);
-        next_k += kTileK;
-    };
     auto issue_act = [&](int i) {
         const int s = i % LS;
         mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kActBytes));
         tma_load_2d(smem + L::kAct + s * L::kActBytes, &tmA, (kb + i) * kTileK, m0, &full[s]);
     };
 
-    const int early = p.prefetch ? min(kEarlyStages, nst) : 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < LS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&wfull[s], 1);
             mbar_init(&afull[s], kDequantWarps);
             mbar_init(&done[s], 1);
         }
@@ -275,9 +242,6 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensor_map(&tmA);
-        // With static weights (set by the caller), start the first weight copies
-        // before waiting for the TMEM allocation and for the previous kernel.
-        for (int i = 0; i < early; ++i) issue_wts();
         grid_launch_dependents();
     }
     if (warp == 1) {
@@ -295,20 +259,17 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         // A stage's slot is free again once the MMAs that read it completed
         // (which also means the dequantisation warps finished reading it).
         if (lane == 0) {
-            grid_dependency_wait();  // anything but static weights may be written by the previous kernel
-            for (int i = 0; i < early; ++i) issue_act(i);
-            while (next_i < nst) {
-                const int i = next_i;
+            grid_dependency_wait();  // the activations may be written by the previous kernel
+            int issued = 0;
+            for (; issued < nst; ++issued) {
+                const int i = issued;
                 if (i >= LS && !wait_phase(&done[i % LS], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
                     break;
-                issue_wts();
                 issue_act(i);
             }
             // Every issued copy must land before the CTA's shared memory is released.
-            for (int i = max(0, next_i - LS); i < next_i; ++i) {
-                drain_phase(&wfull[i % LS], static_cast<uint32_t>(i / LS) & 1u);
+            for (int i = max(0, issued - LS); i < issued; ++i)
                 drain_phase(&full[i % LS], static_cast<uint32_t>(i / LS) & 1u);
-            }
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -317,8 +278,7 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             const uint64_t bdesc0 = smem_desc_k_sw128(smem_addr(smem + L::kAct));
             for (int i = 0; i < nst; ++i) {
                 const int s = i % LS;
-                // The stage's dequantised weights (afull), then its activation tile (full):
-                // the dequantisation warps only wait for the small int4 and scale copies.
+                // The stage's dequantised weights (afull), then its activation tile (full).
                 if (!wait_phase(&afull[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
                 if (!wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
                 tc_fence_after_sync();
@@ -343,31 +303,56 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         const int n = nt * kTileN + j;
         const bool col_ok = n < p.N;
         const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
+        // Codes and scales of this thread's stages (i = grp, grp + DQ, ...) are
+        // loaded two of its stages ahead into registers. kk is the first k of
+        // the thread's 32-deep chunk in the next stage to load, gk = floor(kk / G).
+        const uint8_t* wcol = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes + h * 2048 + j * 16;
+        const __half* scol = p.sc[expert] + (col_ok ? n : 0);
+        const bool one_group = (p.G % kTileK) == 0;  // a 64-deep stage lies inside one scale group
+        int li = grp;
+        int kk = (kb + grp) * kTileK + 32 * h;
+        int gk = kk / p.G;
+        auto load_next = [&](uint4& r, __half (&sv)[4]) {
+            if (li < nst) {
+                r = ld_nc_v4(wcol + static_cast<int64_t>(kb + li) * kRawBytes);
+                if (one_group) {
+                    const __half v = col_ok ? __ldg(scol + static_cast<int64_t>(min(gk, p.ngroups - 1)) * p.N)
+                                            : __float2half(0.f);
+                    sv[0] = sv[1] = sv[2] = sv[3] = v;
+                } else {
+                    const int rem = kk - gk * p.G;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        int g = gk, r2 = rem + 8 * q;
+                        while (r2 >= p.G) {
+                            r2 -= p.G;
+                            ++g;
+                        }
+                        sv[q] = col_ok ? __ldg(scol + static_cast<int64_t>(min(g, p.ngroups - 1)) * p.N)
+                                       : __float2half(0.f);
+                    }
+                }
+            } else {
+                r = make_uint4(0u, 0u, 0u, 0u);
+                sv[0] = sv[1] = sv[2] = sv[3] = __float2half(0.f);
+            }
+            li += DQ;
+            kk += kTileK * DQ;
+            while ((gk + 1) * p.G <= kk) ++gk;
+        };
+        if (!p.prefetch) grid_dependency_wait();  // weights and scales may come from the previous kernel
+        uint4 r0, r1;
+        __half s0[4], s1[4];
+        load_next(r0, s0);
+        load_next(r1, s1);
         for (int i = grp; i < nst; i += DQ) {
             const int s = i % LS;
-            if (!warp_wait_phase(&wfull[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
-            const uint4 raw =
-                *reinterpret_cast<const uint4*>(smem + L::kRaw + s * kRawBytes + h * 2048 + j * 16);
-            const int2 info = stage_info[s];
-            const __half* srow = reinterpret_cast<const __half*>(smem + L::kScale + s * kMaxScaleRows * kScaleRowBytes);
-            const int last = info.y - 1;
-            __half sv[4];
-            if (p.scale_mode == 0) {
-                const __half v = srow[j];
-                sv[0] = sv[1] = sv[2] = sv[3] = v;
-            } else if (p.scale_mode == 1) {
-                const __half v = srow[min(h, last) * kTileN + j];
-                sv[0] = sv[1] = sv[2] = sv[3] = v;
-            } else if (p.scale_mode == 2) {
-                const __half v0 = srow[min(2 * h, last) * kTileN + j];
-                const __half v1 = srow[min(2 * h + 1, last) * kTileN + j];
-                sv[0] = sv[1] = v0;
-                sv[2] = sv[3] = v1;
-            } else {
-                const int k0 = (kb + i) * kTileK + 32 * h;
+            const uint4 raw = r0;
+            const __half sv[4] = {s0[0], s0[1], s0[2], s0[3]};
+            r0 = r1;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) sv[q] = srow[min((k0 + 8 * q) / p.G - info.x, last) * kTileN + j];
-            }
+            for (int q = 0; q < 4; ++q) s0[q] = s1[q];
+            load_next(r1, s1);
             uint32_t v[16];
             {
                 const uint4 o0 = dequant_word(raw.x, __half2half2(sv[0]));
@@ -539,7 +524,7 @@ Variant make_variant() {
 // <token tile, ring stages, TMEM columns, CTAs per SM, dequantisation groups>
 const Variant kVariants[] = {
     make_variant<16, 7, 256, 2, 1>(), make_variant<32, 7, 256, 2, 1>(), make_variant<64, 6, 256, 2, 1>(),
-    make_variant<128, 4, 256, 2, 1>(), make_variant<256, 5, 512, 1, 2>(),
+    make_variant<128, 4, 256, 2, 1>(), make_variant<256, 6, 512, 1, 2>(),
 };
 
 const Variant& variant_for(int bn) {
@@ -609,24 +594,6 @@ int check_shape(int64_t N, int64_t K, int64_t G) {
     if (N % 8 || K % 8 || G % 16) return W4A16_ERR_UNSUPPORTED;
     if (N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
     return W4A16_OK;
-}
-
-void fill_scale_plan(Params& p) {
-    const int G = p.G;
-    if (G % 64 == 0) {
-        p.scale_mode = 0;
-        p.scale_rows = 1;
-    } else if (G == 32) {
-        p.scale_mode = 1;
-        p.scale_rows = 2;
-    } else if (G == 16) {
-        p.scale_mode = 2;
-        p.scale_rows = 4;
-    } else {
-        p.scale_mode = 3;
-        p.scale_rows = 64 / G + 2;
-    }
-    if (p.scale_rows > kMaxScaleRows) p.scale_rows = kMaxScaleRows;
 }
 
 struct Plan {
@@ -851,7 +818,6 @@ extern "C" int w4a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt_dev, const 
     p.splits = plan.splits;
     p.grouped = 0;
     p.prefetch = static_weights_enabled() ? 1 : 0;
-    fill_scale_plan(p);
 
     CUtensorMap map;
     rc = make_act_map(&map, A_dev, M, K, plan.bn);
@@ -900,7 +866,6 @@ extern "C" int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const*
     p.splits = 1;
     p.grouped = 1;
     p.prefetch = 0;  // expert weights are read only after the offsets, which follow the wait
-    fill_scale_plan(p);
 
     CUtensorMap map;
     rc = make_act_map(&map, A_dev, total_rows, K, plan.bn);
