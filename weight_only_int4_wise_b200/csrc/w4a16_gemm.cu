@@ -54,6 +54,7 @@ constexpr int kTileK = 64;                  // K per pipeline stage
 constexpr int kRawBytes = 4096;             // int4 codes of one 128 x 64 tile
 constexpr int kSlotCols = kTileK / 2;       // TMEM columns of one dequantised 128 x 64 fp16 tile
 constexpr int kDequantWarps = 8;           // one group: 4 TMEM lane quadrants x 2 halves of a stage
+constexpr int kAhead = 2;                  // stages of its own a dequantising thread loads ahead
 // Threads of a CTA with DQ dequantisation groups (each group takes every
 // DQ-th stage, so DQ groups keep DQ stages in flight).
 __host__ __device__ constexpr int threads_for(int dq) { return (2 + kDequantWarps * dq) * 32; }
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         const bool col_ok = n < p.N;
         const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
         // Codes and scales of this thread's stages (i = grp, grp + DQ, ...) are
-        // loaded two of its stages ahead into registers. kk is the first k of
+        // loaded kAhead of its stages ahead into registers. kk is the first k of
         // the thread's 32-deep chunk in the next stage to load, gk = floor(kk / G).
         const uint8_t* wcol = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes + h * 2048 + j * 16;
         const __half* scol = p.sc[expert] + (col_ok ? n : 0);
@@ -341,18 +342,21 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             while ((gk + 1) * p.G <= kk) ++gk;
         };
         if (!p.prefetch) grid_dependency_wait();  // weights and scales may come from the previous kernel
-        uint4 r0, r1;
-        __half s0[4], s1[4];
-        load_next(r0, s0);
-        load_next(r1, s1);
+        uint4 rq[kAhead];
+        __half sq[kAhead][4];
+#pragma unroll
+        for (int d = 0; d < kAhead; ++d) load_next(rq[d], sq[d]);
         for (int i = grp; i < nst; i += DQ) {
             const int s = i % LS;
-            const uint4 raw = r0;
-            const __half sv[4] = {s0[0], s0[1], s0[2], s0[3]};
-            r0 = r1;
+            const uint4 raw = rq[0];
+            const __half sv[4] = {sq[0][0], sq[0][1], sq[0][2], sq[0][3]};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) s0[q] = s1[q];
-            load_next(r1, s1);
+            for (int d = 0; d + 1 < kAhead; ++d) {  // (a fixed rotation: the ring stays in registers)
+                rq[d] = rq[d + 1];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) sq[d][q] = sq[d + 1][q];
+            }
+            load_next(rq[kAhead - 1], sq[kAhead - 1]);
             uint32_t v[16];
             {
                 const uint4 o0 = dequant_word(raw.x, __half2half2(sv[0]));
@@ -364,10 +368,7 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
                 v[8] = o2.x; v[9] = o2.y; v[10] = o2.z; v[11] = o2.w;
                 v[12] = o3.x; v[13] = o3.y; v[14] = o3.z; v[15] = o3.w;
             }
-            if (!col_ok) {
-#pragma unroll
-                for (int t = 0; t < 16; ++t) v[t] = 0u;
-            }
+            // (Columns past N hold code 0 in the tiled layout and get scale 0: v is 0.)
             if (i >= LS && !warp_wait_phase(&done[s], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
                 break;
             tc_fence_after_sync();
