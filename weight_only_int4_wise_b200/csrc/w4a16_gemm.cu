@@ -58,6 +58,7 @@ constexpr int kAhead = 2;                  // stages of its own a dequantising t
 // Threads of a CTA with DQ dequantisation groups (each group takes every
 // DQ-th stage, so DQ groups keep DQ stages in flight).
 __host__ __device__ constexpr int threads_for(int dq) { return (2 + kDequantWarps * dq) * 32; }
+static_assert(threads_for(3) <= 1024, "at most three dequantisation groups fit a CTA");
 constexpr long long kTimeoutCycles = 4000000000ll;  // about 2 s per wait at the boost clock
 
 struct Params {
@@ -520,12 +521,13 @@ Variant make_variant() {
 }
 
 // Token tiles and their pipeline depths: small tiles keep two CTAs per SM; the
-// 256-row tile (one CTA per SM, MMAs of N = 256) runs two dequantisation
-// groups so that decoding two stages at once keeps pace with the tensor core.
+// 256-row tile (one CTA per SM) runs three dequantisation groups (832
+// threads) so that decoding three stages at once keeps pace with the tensor
+// core, which matters most for expert tiles of about 128 rows.
 // <token tile, ring stages, TMEM columns, CTAs per SM, dequantisation groups>
 const Variant kVariants[] = {
     make_variant<16, 7, 256, 2, 1>(), make_variant<32, 7, 256, 2, 1>(), make_variant<64, 6, 256, 2, 1>(),
-    make_variant<128, 4, 256, 2, 1>(), make_variant<256, 6, 512, 1, 2>(),
+    make_variant<128, 4, 256, 2, 1>(), make_variant<256, 6, 512, 1, 3>(),
 };
 
 const Variant& variant_for(int bn) {
