@@ -86,7 +86,7 @@ struct Layout {
     static constexpr int kActBytes = BN * 128;
     static constexpr int kAct = 0;
     static constexpr int kBar = kAct + LS * kActBytes;
-    static constexpr int kNumBars = 3 * LS + 1;
+    static constexpr int kNumBars = LS + LS / 2 + LS + 1;  // full, afull (per stage pair), done, accfull
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base, abort flag, tile info
     static constexpr int kTotal = kMisc + 32;
     static constexpr int kAlloc = kTotal + 1024;       // slack for aligning the base to 1024
@@ -97,6 +97,7 @@ struct Layout {
                   "TMEM allocations are powers of two");
     static_assert(kRedBytes <= kBar, "split-K buffer must fit in the activation ring");
     static_assert((kActBytes % 1024) == 0, "activation tiles need 1024-byte alignment");
+    static_assert((LS % 2) == 0, "the MMA thread takes the ring two stages at a time");
 };
 
 __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
@@ -170,8 +171,8 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
     uint8_t* smem = smem_raw + ((1024u - (base_addr & 1023u)) & 1023u);
 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);   // stage's copies landed
-    uint64_t* afull = full + LS;                                     // stage's TMEM weights written
-    uint64_t* done = afull + LS;                                     // stage's MMAs completed
+    uint64_t* afull = full + LS;                                     // stage pair ready for the MMAs
+    uint64_t* done = afull + LS / 2;                                 // stage's MMAs completed
     uint64_t* accfull = done + LS;                                   // accumulator complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
@@ -237,9 +238,9 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
     if (threadIdx.x == 0) {
         for (int s = 0; s < LS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&afull[s], kDequantWarps);
             mbar_init(&done[s], 1);
         }
+        for (int q = 0; q < LS / 2; ++q) mbar_init(&afull[q], 2 * kDequantWarps);
         mbar_init(accfull, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -277,20 +278,28 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
+            // One barrier per pair of stages covers both operands of both stages:
+            // the dequantised weights and, through each group's first warp, the
+            // landed activation tiles. (Each wait costs the single issuing thread
+            // about as long as an MMA, so it is paid once per eight MMAs.)
             const uint64_t bdesc0 = smem_desc_k_sw128(smem_addr(smem + L::kAct));
-            for (int i = 0; i < nst; ++i) {
-                const int s = i % LS;
-                // The stage's dequantised weights (afull), then its activation tile (full).
-                if (!wait_phase(&afull[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
-                if (!wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag)) break;
+            for (int i = 0; i < nst; i += 2) {
+                const int q = i >> 1;
+                if (!wait_phase(&afull[q % (LS / 2)], static_cast<uint32_t>(q / (LS / 2)) & 1u, abort_flag)) break;
                 tc_fence_after_sync();
-                const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((s * L::kActBytes) >> 4);
-                const uint32_t a0 = tmem_ring + s * kSlotCols;
-                mma_f16_ts(tmem_acc, a0, bdesc, idesc, i > 0 ? 1u : 0u);
-                mma_f16_ts(tmem_acc, a0 + 8, bdesc + 2, idesc, 1u);
-                mma_f16_ts(tmem_acc, a0 + 16, bdesc + 4, idesc, 1u);
-                mma_f16_ts(tmem_acc, a0 + 24, bdesc + 6, idesc, 1u);
-                mma_commit(&done[s]);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (i + t < nst) {
+                        const int s = (i + t) % LS;
+                        const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((s * L::kActBytes) >> 4);
+                        const uint32_t a0 = tmem_ring + s * kSlotCols;
+                        mma_f16_ts(tmem_acc, a0, bdesc, idesc, (i + t) > 0 ? 1u : 0u);
+                        mma_f16_ts(tmem_acc, a0 + 8, bdesc + 2, idesc, 1u);
+                        mma_f16_ts(tmem_acc, a0 + 16, bdesc + 4, idesc, 1u);
+                        mma_f16_ts(tmem_acc, a0 + 24, bdesc + 6, idesc, 1u);
+                        mma_commit(&done[s]);
+                    }
+                }
             }
             mma_commit(accfull);  // fires once every MMA issued above has completed
         }
@@ -376,8 +385,13 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             tmem_st_32x32b_x16(tmem_ring + tlane + s * kSlotCols + h * 16, v);
             tmem_st_wait();
             tc_fence_before_sync();
+            // The group's first warp also sees the stage's activation tile land,
+            // so that the MMA thread waits on one barrier per stage pair. The
+            // last stage of an odd count arrives for its missing partner too.
+            if ((dw & 7) == 0 && !warp_wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag))
+                break;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&afull[s]);
+            if (lane == 0) mbar_arrive_cnt(&afull[(i >> 1) % (LS / 2)], ((i & 1) == 0 && i + 1 == nst) ? 2u : 1u);
         }
 
         // -------------------------------------------------- epilogue
@@ -526,7 +540,7 @@ Variant make_variant() {
 // core, which matters most for expert tiles of about 128 rows.
 // <token tile, ring stages, TMEM columns, CTAs per SM, dequantisation groups>
 const Variant kVariants[] = {
-    make_variant<16, 7, 256, 2, 1>(), make_variant<32, 7, 256, 2, 1>(), make_variant<64, 6, 256, 2, 1>(),
+    make_variant<16, 6, 256, 2, 1>(), make_variant<32, 6, 256, 2, 1>(), make_variant<64, 6, 256, 2, 1>(),
     make_variant<128, 4, 256, 2, 1>(), make_variant<256, 6, 512, 1, 3>(),
 };
 
