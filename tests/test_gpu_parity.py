@@ -58,10 +58,10 @@ def test_repack_bit_exact(o, K, N):
 
 # --------------------------------------------------------------- small GEMMs
 
-def run_dense(o, M, K, N, G, seed, a_scale=1.0):
+def run_dense(o, M, K, N, G, seed, a_scale=1.0, pad=64):
     c = workloads.dense(M, K, N, G, seed, a_scale=a_scale)
     _, wt = device_weights(c.q)
-    flat, C, pad = guarded_output(M, N)
+    flat, C, pad = guarded_output(M, N, pad)
     w.gemm(dev(c.A), wt, dev(c.S), N, G, out=C)
     torch.cuda.synchronize()
     got = C.cpu().numpy()
@@ -90,6 +90,12 @@ def test_ragged_rows(o, M):
 def test_shapes_and_group_sizes(o, K, N, G):
     for M in (1, 8, 40):
         run_dense(o, M, K, N, G, seed=K * 7 + N + G + M)
+
+
+@pytest.mark.parametrize("M", [1, 17, 300])
+def test_output_rows_off_16_byte_boundaries(o, M):
+    # C starts 2 bytes past a 16-byte boundary: the row stores cannot be 16-byte vectors
+    run_dense(o, M, 200, 392, 64, seed=500 + M, pad=65)
 
 
 def test_large_activations_stay_in_tolerance(o):

@@ -74,6 +74,7 @@ struct Params {
     int32_t splits;     // CTAs along K (cluster size along x)
     int32_t grouped;
     int32_t prefetch;   // weights/scales may be read before the previous kernel finishes
+    int32_t vec_out;    // C rows start on 16-byte boundaries (16-byte output stores)
 };
 
 // One ring of LS stages. Stage s owns, in shared memory, an activation tile
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
     uint64_t* accfull = done + LS;                                   // accumulator complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-    int* tile_info = reinterpret_cast<int*>(smem + L::kMisc + 8);  // has_tile, expert, m0, rows
+    int* tile_info = reinterpret_cast<int*>(smem + L::kMisc + 8);  // has_tile, expert, m0, rows, staged
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -402,20 +403,19 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         grid_dependency_wait();  // the output may still be read by the previous kernel
         const int aborted = __shfl_sync(0xffffffffu, *abort_flag, 0);
         const bool have_acc = !aborted && nst > 0;
+        if (dw == 0 && lane == 0) tile_info[4] = have_acc ? 1 : 0;
         if (p.splits == 1) {
+            // Stage the fp16 tile, row-major [token][128 columns], in the idle
+            // activation ring (every copy into it was consumed by a completed
+            // MMA), so that the global stores below are whole 16-byte vectors.
             if (have_acc) {
-                __half* cbase = p.C + static_cast<int64_t>(m0) * p.N + n;
+                __half* stile = reinterpret_cast<__half*>(smem + L::kAct);
                 for (int c = h + 2 * grp; c < n_mma / 16; c += 2 * DQ) {
                     uint32_t v[16];
                     tmem_ld_32x32b_x16(tmem_acc + tlane + c * 16, v);
                     tmem_ld_wait();
-                    if (col_ok) {
 #pragma unroll
-                        for (int t = 0; t < 16; ++t) {
-                            const int r = c * 16 + t;
-                            if (r < rows) cbase[static_cast<int64_t>(r) * p.N] = __float2half_rn(__uint_as_float(v[t]));
-                        }
-                    }
+                    for (int t = 0; t < 16; ++t) stile[(c * 16 + t) * kTileN + j] = __float2half_rn(__uint_as_float(v[t]));
                 }
             }
         } else {
@@ -440,6 +440,23 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
     if (warp == 1) {
         tc_fence_after_sync();
         tmem_dealloc(tmem_acc, TMEM_COLS);
+    }
+
+    if (p.splits == 1 && tile_info[4]) {
+        // Row r of the tile is 16 chunks of 8 columns; a warp writes two rows
+        // per instruction.
+        const __half* stile = reinterpret_cast<const __half*>(smem + L::kAct);
+        const int n0 = nt * kTileN;
+        for (int o = threadIdx.x; o < rows * 16; o += static_cast<int>(blockDim.x)) {
+            const int r = o >> 4;
+            const int cc = (o & 15) * 8;
+            __half* dst = p.C + static_cast<int64_t>(m0 + r) * p.N + n0 + cc;
+            if (p.vec_out && n0 + cc + 8 <= p.N) {
+                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(stile + r * kTileN + cc);
+            } else {
+                for (int e = 0; e < 8 && n0 + cc + e < p.N; ++e) dst[e] = stile[r * kTileN + cc + e];
+            }
+        }
     }
 
     if (p.splits > 1) {
@@ -835,6 +852,7 @@ extern "C" int w4a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt_dev, const 
     p.splits = plan.splits;
     p.grouped = 0;
     p.prefetch = static_weights_enabled() ? 1 : 0;
+    p.vec_out = (N % 8) == 0 && aligned16(C_dev);
 
     CUtensorMap map;
     rc = make_act_map(&map, A_dev, M, K, plan.bn);
@@ -882,6 +900,7 @@ extern "C" int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const*
     p.E = static_cast<int32_t>(E);
     p.splits = 1;
     p.grouped = 1;
+    p.vec_out = (N % 8) == 0 && aligned16(C_dev);
     p.prefetch = 0;  // expert weights are read only after the offsets, which follow the wait
 
     CUtensorMap map;
