@@ -53,12 +53,12 @@ constexpr int kTileN = 128;                 // weight columns per CTA (MMA M)
 constexpr int kTileK = 64;                  // K per pipeline stage
 constexpr int kRawBytes = 4096;             // int4 codes of one 128 x 64 tile
 constexpr int kSlotCols = kTileK / 2;       // TMEM columns of one dequantised 128 x 64 fp16 tile
-constexpr int kDequantWarps = 8;           // one group: 4 TMEM lane quadrants x 2 halves of a stage
+constexpr int kGroupWarps = 4;             // one dequantisation group: the 4 TMEM lane quadrants
 constexpr int kAhead = 2;                  // stages of its own a dequantising thread loads ahead
 // Threads of a CTA with DQ dequantisation groups (each group takes every
 // DQ-th stage, so DQ groups keep DQ stages in flight).
-__host__ __device__ constexpr int threads_for(int dq) { return (2 + kDequantWarps * dq) * 32; }
-static_assert(threads_for(3) <= 1024, "at most three dequantisation groups fit a CTA");
+__host__ __device__ constexpr int threads_for(int dq) { return (2 + kGroupWarps * dq) * 32; }
+static_assert(threads_for(4) <= 1024, "the 256-row tile's four dequantisation groups fit a CTA");
 constexpr long long kTimeoutCycles = 4000000000ll;  // about 2 s per wait at the boost clock
 
 struct Params {
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             mbar_init(&full[s], 1);
             mbar_init(&done[s], 1);
         }
-        for (int q = 0; q < LS / 2; ++q) mbar_init(&afull[q], 2 * kDequantWarps);
+        for (int q = 0; q < LS / 2; ++q) mbar_init(&afull[q], 2 * kGroupWarps);
         mbar_init(accfull, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -308,88 +308,99 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
     } else {
         // ------------------------------------------------------ dequant + epilogue
         const int dw = warp - 2;
-        const int grp = dw >> 3;          // dequantisation group: stages grp, grp + DQ, ...
-        const int h = (dw >> 2) & 1;      // which 32-deep half of the stage
+        const int grp = dw >> 2;          // dequantisation group: stages grp, grp + DQ, ...
         const int quad = warp & 3;        // TMEM lane quadrant this warp may access
         const int j = quad * 32 + lane;   // weight column inside the tile = TMEM lane
         const int n = nt * kTileN + j;
         const bool col_ok = n < p.N;
         const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
         // Codes and scales of this thread's stages (i = grp, grp + DQ, ...) are
-        // loaded kAhead of its stages ahead into registers. kk is the first k of
-        // the thread's 32-deep chunk in the next stage to load, gk = floor(kk / G).
-        const uint8_t* wcol = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes + h * 2048 + j * 16;
+        // loaded kAhead of its stages ahead into registers: the two 16-byte
+        // halves (k 0..31 and 32..63) of the column's stage, and one scale per
+        // 8-deep word (as pairs: words 2q, 2q+1 in one half2). kk is the first k
+        // of the next stage to load, gk = floor(kk / G).
+        const uint8_t* wcol = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes + j * 16;
         const __half* scol = p.sc[expert] + (col_ok ? n : 0);
         const bool one_group = (p.G % kTileK) == 0;  // a 64-deep stage lies inside one scale group
         int li = grp;
-        int kk = (kb + grp) * kTileK + 32 * h;
+        int kk = (kb + grp) * kTileK;
         int gk = kk / p.G;
-        auto load_next = [&](uint4& r, __half (&sv)[4]) {
+        auto load_next = [&](uint4 (&r)[2], __half2 (&sv)[4]) {
             if (li < nst) {
-                r = ld_nc_v4(wcol + static_cast<int64_t>(kb + li) * kRawBytes);
+                const uint8_t* src = wcol + static_cast<int64_t>(kb + li) * kRawBytes;
+                r[0] = ld_nc_v4(src);
+                r[1] = ld_nc_v4(src + kRawBytes / 2);
                 if (one_group) {
                     const __half v = col_ok ? __ldg(scol + static_cast<int64_t>(min(gk, p.ngroups - 1)) * p.N)
                                             : __float2half(0.f);
-                    sv[0] = sv[1] = sv[2] = sv[3] = v;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) sv[q] = __half2half2(v);
                 } else {
                     const int rem = kk - gk * p.G;
+                    __half w[8];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
+                    for (int q = 0; q < 8; ++q) {
                         int g = gk, r2 = rem + 8 * q;
                         while (r2 >= p.G) {
                             r2 -= p.G;
                             ++g;
                         }
-                        sv[q] = col_ok ? __ldg(scol + static_cast<int64_t>(min(g, p.ngroups - 1)) * p.N)
-                                       : __float2half(0.f);
+                        w[q] = col_ok ? __ldg(scol + static_cast<int64_t>(min(g, p.ngroups - 1)) * p.N)
+                                      : __float2half(0.f);
                     }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) sv[q] = __halves2half2(w[2 * q], w[2 * q + 1]);
                 }
             } else {
-                r = make_uint4(0u, 0u, 0u, 0u);
-                sv[0] = sv[1] = sv[2] = sv[3] = __float2half(0.f);
+                r[0] = r[1] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) sv[q] = __float2half2_rn(0.f);
             }
             li += DQ;
             kk += kTileK * DQ;
             while ((gk + 1) * p.G <= kk) ++gk;
         };
         if (!p.prefetch) grid_dependency_wait();  // weights and scales may come from the previous kernel
-        uint4 rq[kAhead];
-        __half sq[kAhead][4];
+        uint4 rq[kAhead][2];
+        __half2 sq[kAhead][4];
 #pragma unroll
         for (int d = 0; d < kAhead; ++d) load_next(rq[d], sq[d]);
         for (int i = grp; i < nst; i += DQ) {
             const int s = i % LS;
-            const uint4 raw = rq[0];
-            const __half sv[4] = {sq[0][0], sq[0][1], sq[0][2], sq[0][3]};
+            const uint32_t raw[8] = {rq[0][0].x, rq[0][0].y, rq[0][0].z, rq[0][0].w,
+                                     rq[0][1].x, rq[0][1].y, rq[0][1].z, rq[0][1].w};
+            __half2 sv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sv[q] = sq[0][q];
 #pragma unroll
             for (int d = 0; d + 1 < kAhead; ++d) {  // (a fixed rotation: the ring stays in registers)
-                rq[d] = rq[d + 1];
+                rq[d][0] = rq[d + 1][0];
+                rq[d][1] = rq[d + 1][1];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) sq[d][q] = sq[d + 1][q];
             }
             load_next(rq[kAhead - 1], sq[kAhead - 1]);
-            uint32_t v[16];
-            {
-                const uint4 o0 = dequant_word(raw.x, __half2half2(sv[0]));
-                const uint4 o1 = dequant_word(raw.y, __half2half2(sv[1]));
-                const uint4 o2 = dequant_word(raw.z, __half2half2(sv[2]));
-                const uint4 o3 = dequant_word(raw.w, __half2half2(sv[3]));
-                v[0] = o0.x; v[1] = o0.y; v[2] = o0.z; v[3] = o0.w;
-                v[4] = o1.x; v[5] = o1.y; v[6] = o1.z; v[7] = o1.w;
-                v[8] = o2.x; v[9] = o2.y; v[10] = o2.z; v[11] = o2.w;
-                v[12] = o3.x; v[13] = o3.y; v[14] = o3.z; v[15] = o3.w;
+            uint32_t v[2][16];  // k 0..31, k 32..63
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const uint4 o = dequant_word(raw[q], (q & 1) ? __high2half2(sv[q >> 1]) : __low2half2(sv[q >> 1]));
+                v[q >> 2][4 * (q & 3)] = o.x;
+                v[q >> 2][4 * (q & 3) + 1] = o.y;
+                v[q >> 2][4 * (q & 3) + 2] = o.z;
+                v[q >> 2][4 * (q & 3) + 3] = o.w;
             }
             // (Columns past N hold code 0 in the tiled layout and get scale 0: v is 0.)
             if (i >= LS && !warp_wait_phase(&done[s], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
                 break;
             tc_fence_after_sync();
-            tmem_st_32x32b_x16(tmem_ring + tlane + s * kSlotCols + h * 16, v);
+            tmem_st_32x32b_x16(tmem_ring + tlane + s * kSlotCols, v[0]);
+            tmem_st_32x32b_x16(tmem_ring + tlane + s * kSlotCols + 16, v[1]);
             tmem_st_wait();
             tc_fence_before_sync();
             // The group's first warp also sees the stage's activation tile land,
             // so that the MMA thread waits on one barrier per stage pair. The
             // last stage of an odd count arrives for its missing partner too.
-            if ((dw & 7) == 0 && !warp_wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag))
+            if ((dw & 3) == 0 && !warp_wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag))
                 break;
             __syncwarp();
             if (lane == 0) mbar_arrive_cnt(&afull[(i >> 1) % (LS / 2)], ((i & 1) == 0 && i + 1 == nst) ? 2u : 1u);
@@ -410,7 +421,7 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             // MMA), so that the global stores below are whole 16-byte vectors.
             if (have_acc) {
                 __half* stile = reinterpret_cast<__half*>(smem + L::kAct);
-                for (int c = h + 2 * grp; c < n_mma / 16; c += 2 * DQ) {
+                for (int c = grp; c < n_mma / 16; c += DQ) {
                     uint32_t v[16];
                     tmem_ld_32x32b_x16(tmem_acc + tlane + c * 16, v);
                     tmem_ld_wait();
@@ -420,7 +431,7 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             }
         } else {
             float* red = reinterpret_cast<float*>(smem + L::kAct);
-            for (int c = h + 2 * grp; c < BN / 16; c += 2 * DQ) {
+            for (int c = grp; c < BN / 16; c += DQ) {
                 uint32_t v[16];
                 if (have_acc && c * 16 < n_mma) {
                     tmem_ld_32x32b_x16(tmem_acc + tlane + c * 16, v);
@@ -552,13 +563,15 @@ Variant make_variant() {
 }
 
 // Token tiles and their pipeline depths: small tiles keep two CTAs per SM; the
-// 256-row tile (one CTA per SM) runs three dequantisation groups (832
-// threads) so that decoding three stages at once keeps pace with the tensor
-// core, which matters most for expert tiles of about 128 rows.
+// 256-row tile (one CTA per SM) runs four dequantisation groups of four warps
+// (576 threads): each group has four stage periods to decode and store its
+// stage. More groups (more warps competing for issue slots, and register
+// spills above five) and fewer groups (too little time per stage) both ran
+// slower on the prefill and grouped-expert shapes.
 // <token tile, ring stages, TMEM columns, CTAs per SM, dequantisation groups>
 const Variant kVariants[] = {
-    make_variant<16, 6, 256, 2, 1>(), make_variant<32, 6, 256, 2, 1>(), make_variant<64, 6, 256, 2, 1>(),
-    make_variant<128, 4, 256, 2, 1>(), make_variant<256, 6, 512, 1, 3>(),
+    make_variant<16, 6, 256, 2, 2>(), make_variant<32, 6, 256, 2, 2>(), make_variant<64, 6, 256, 2, 2>(),
+    make_variant<128, 4, 256, 2, 2>(), make_variant<256, 6, 512, 1, 4>(),
 };
 
 const Variant& variant_for(int bn) {
