@@ -55,6 +55,7 @@ constexpr int kRawBytes = 4096;             // int4 codes of one 128 x 64 tile
 constexpr int kSlotCols = kTileK / 2;       // TMEM columns of one dequantised 128 x 64 fp16 tile
 constexpr int kGroupWarps = 4;             // one dequantisation group: the 4 TMEM lane quadrants
 constexpr int kAhead = 2;                  // stages of its own a dequantising thread loads ahead
+constexpr int kPrefetchStages = 12;        // int4 tile stages the producer pulls into L2 ahead of use
 // Threads of a CTA with DQ dequantisation groups (each group takes every
 // DQ-th stage, so DQ groups keep DQ stages in flight).
 __host__ __device__ constexpr int threads_for(int dq) { return (2 + kGroupWarps * dq) * 32; }
@@ -264,12 +265,19 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         // (which also means the dequantisation warps finished reading it).
         if (lane == 0) {
             grid_dependency_wait();  // the activations may be written by the previous kernel
+            // The int4 tile of a stage is one contiguous 4 KB block: pull it into
+            // L2 kPrefetchStages ahead, so that the dequantising threads' own
+            // loads (issued only kAhead of their stages ahead) find it there.
+            const uint8_t* wtile = p.wt[expert] + (static_cast<int64_t>(nt) * p.KT + kb) * kRawBytes;
+            for (int i = 0; i < min(nst, kPrefetchStages); ++i) bulk_prefetch_l2(wtile + static_cast<int64_t>(i) * kRawBytes, kRawBytes);
             int issued = 0;
             for (; issued < nst; ++issued) {
                 const int i = issued;
                 if (i >= LS && !wait_phase(&done[i % LS], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
                     break;
                 issue_act(i);
+                if (i + kPrefetchStages < nst)
+                    bulk_prefetch_l2(wtile + static_cast<int64_t>(i + kPrefetchStages) * kRawBytes, kRawBytes);
             }
             // Every issued copy must land before the CTA's shared memory is released.
             for (int i = max(0, issued - LS); i < issued; ++i)
