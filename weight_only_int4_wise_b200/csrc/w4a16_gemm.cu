@@ -369,25 +369,12 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             while ((gk + 1) * p.G <= kk) ++gk;
         };
         if (!p.prefetch) grid_dependency_wait();  // weights and scales may come from the previous kernel
-        uint4 rq[kAhead][2];
-        __half2 sq[kAhead][4];
-#pragma unroll
-        for (int d = 0; d < kAhead; ++d) load_next(rq[d], sq[d]);
-        for (int i = grp; i < nst; i += DQ) {
+        // One stage: decode the codes and scales held in (r, sv), refill them
+        // with the thread's stage kAhead of its stages later, store the fp16
+        // weights into the stage's TMEM slot and arrive. False when aborting.
+        auto stage = [&](int i, uint4 (&r)[2], __half2 (&sv)[4]) -> bool {
             const int s = i % LS;
-            const uint32_t raw[8] = {rq[0][0].x, rq[0][0].y, rq[0][0].z, rq[0][0].w,
-                                     rq[0][1].x, rq[0][1].y, rq[0][1].z, rq[0][1].w};
-            __half2 sv[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) sv[q] = sq[0][q];
-#pragma unroll
-            for (int d = 0; d + 1 < kAhead; ++d) {  // (a fixed rotation: the ring stays in registers)
-                rq[d][0] = rq[d + 1][0];
-                rq[d][1] = rq[d + 1][1];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) sq[d][q] = sq[d + 1][q];
-            }
-            load_next(rq[kAhead - 1], sq[kAhead - 1]);
+            const uint32_t raw[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
             uint32_t v[2][16];  // k 0..31, k 32..63
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -397,9 +384,10 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
                 v[q >> 2][4 * (q & 3) + 2] = o.z;
                 v[q >> 2][4 * (q & 3) + 3] = o.w;
             }
+            load_next(r, sv);
             // (Columns past N hold code 0 in the tiled layout and get scale 0: v is 0.)
             if (i >= LS && !warp_wait_phase(&done[s], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
-                break;
+                return false;
             tc_fence_after_sync();
             tmem_st_32x32b_x16(tmem_ring + tlane + s * kSlotCols, v[0]);
             tmem_st_32x32b_x16(tmem_ring + tlane + s * kSlotCols + 16, v[1]);
@@ -409,9 +397,22 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             // so that the MMA thread waits on one barrier per stage pair. The
             // last stage of an odd count arrives for its missing partner too.
             if ((dw & 3) == 0 && !warp_wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag))
-                break;
+                return false;
             __syncwarp();
             if (lane == 0) mbar_arrive_cnt(&afull[(i >> 1) % (LS / 2)], ((i & 1) == 0 && i + 1 == nst) ? 2u : 1u);
+            return true;
+        };
+        // kAhead = 2 register slots, used alternately: a stage's codes stay in
+        // the registers they were loaded into (moving a register whose load is
+        // still in flight would wait for that load).
+        static_assert(kAhead == 2, "the stage loop below alternates two register slots");
+        uint4 rq0[2], rq1[2];
+        __half2 sq0[4], sq1[4];
+        load_next(rq0, sq0);
+        load_next(rq1, sq1);
+        for (int i = grp; i < nst; i += 2 * DQ) {
+            if (!stage(i, rq0, sq0)) break;
+            if (i + DQ < nst && !stage(i + DQ, rq1, sq1)) break;
         }
 
         // -------------------------------------------------- epilogue
