@@ -92,6 +92,12 @@ def test_shapes_and_group_sizes(o, K, N, G):
         run_dense(o, M, K, N, G, seed=K * 7 + N + G + M)
 
 
+@pytest.mark.parametrize("K,N,G", [(520, 264, 48), (1032, 136, 16), (200, 392, 80)])
+def test_group_sizes_not_multiple_of_64_on_the_largest_tile(o, K, N, G):
+    # 300 rows: one full 256-row tile and a ragged one; per-word scales in a stage
+    run_dense(o, 300, K, N, G, seed=K + N + G)
+
+
 @pytest.mark.parametrize("M", [1, 17, 300])
 def test_output_rows_off_16_byte_boundaries(o, M):
     # C starts 2 bytes past a 16-byte boundary: the row stores cannot be 16-byte vectors

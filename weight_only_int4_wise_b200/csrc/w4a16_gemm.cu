@@ -164,10 +164,12 @@ __device__ __forceinline__ void warp_drain_phase(uint64_t* bar, uint32_t parity)
     if (ok) mbar_try_wait(bar, parity);
 }
 
-template <int BN, int LS, int TMEM_COLS, int MINB, int DQ>
+// OG: G is a multiple of 64, so a stage lies inside one scale group.
+template <int BN, int LS, int TMEM_COLS, int MINB, int DQ, bool OG>
 __global__ void __launch_bounds__(threads_for(DQ), MINB)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ Params p) {
     using L = Layout<BN, LS, TMEM_COLS>;
+    constexpr int kScales = OG ? 1 : 8;  // scale registers per stage and thread
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base_addr = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (base_addr & 1023u)) & 1023u);
@@ -324,28 +326,26 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
         // Codes and scales of this thread's stages (i = grp, grp + DQ, ...) are
         // loaded kAhead of its stages ahead into registers: the two 16-byte
-        // halves (k 0..31 and 32..63) of the column's stage, and one scale per
-        // 8-deep word (as pairs: words 2q, 2q+1 in one half2). kk is the first k
-        // of the next stage to load, gk = floor(kk / G).
+        // halves (k 0..31 and 32..63) of the column's stage and its scales (one
+        // when G is a multiple of 64, else one per 8-deep word). Loaded values
+        // are left exactly as loaded until the stage is decoded: any instruction
+        // that reads a register whose load is in flight waits for that load.
+        // kk is the first k of the next stage to load, gk = floor(kk / G).
+        // (A padded column past N reads column 0's scales; its codes are 0.)
         const uint8_t* wcol = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes + j * 16;
         const __half* scol = p.sc[expert] + (col_ok ? n : 0);
-        const bool one_group = (p.G % kTileK) == 0;  // a 64-deep stage lies inside one scale group
         int li = grp;
         int kk = (kb + grp) * kTileK;
         int gk = kk / p.G;
-        auto load_next = [&](uint4 (&r)[2], __half2 (&sv)[4]) {
+        auto load_next = [&](uint4 (&r)[2], __half (&sv)[kScales]) {
             if (li < nst) {
                 const uint8_t* src = wcol + static_cast<int64_t>(kb + li) * kRawBytes;
                 r[0] = ld_nc_v4(src);
                 r[1] = ld_nc_v4(src + kRawBytes / 2);
-                if (one_group) {
-                    const __half v = col_ok ? __ldg(scol + static_cast<int64_t>(min(gk, p.ngroups - 1)) * p.N)
-                                            : __float2half(0.f);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) sv[q] = __half2half2(v);
+                if constexpr (OG) {
+                    sv[0] = __ldg(scol + static_cast<int64_t>(min(gk, p.ngroups - 1)) * p.N);
                 } else {
                     const int rem = kk - gk * p.G;
-                    __half w[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         int g = gk, r2 = rem + 8 * q;
@@ -353,16 +353,13 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
                             r2 -= p.G;
                             ++g;
                         }
-                        w[q] = col_ok ? __ldg(scol + static_cast<int64_t>(min(g, p.ngroups - 1)) * p.N)
-                                      : __float2half(0.f);
+                        sv[q] = __ldg(scol + static_cast<int64_t>(min(g, p.ngroups - 1)) * p.N);
                     }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) sv[q] = __halves2half2(w[2 * q], w[2 * q + 1]);
                 }
             } else {
                 r[0] = r[1] = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) sv[q] = __float2half2_rn(0.f);
+                for (int q = 0; q < kScales; ++q) sv[q] = __float2half(0.f);
             }
             li += DQ;
             kk += kTileK * DQ;
@@ -372,13 +369,13 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         // One stage: decode the codes and scales held in (r, sv), refill them
         // with the thread's stage kAhead of its stages later, store the fp16
         // weights into the stage's TMEM slot and arrive. False when aborting.
-        auto stage = [&](int i, uint4 (&r)[2], __half2 (&sv)[4]) -> bool {
+        auto stage = [&](int i, uint4 (&r)[2], __half (&sv)[kScales]) -> bool {
             const int s = i % LS;
             const uint32_t raw[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
             uint32_t v[2][16];  // k 0..31, k 32..63
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const uint4 o = dequant_word(raw[q], (q & 1) ? __high2half2(sv[q >> 1]) : __low2half2(sv[q >> 1]));
+                const uint4 o = dequant_word(raw[q], __half2half2(sv[OG ? 0 : q]));
                 v[q >> 2][4 * (q & 3)] = o.x;
                 v[q >> 2][4 * (q & 3) + 1] = o.y;
                 v[q >> 2][4 * (q & 3) + 2] = o.z;
@@ -407,7 +404,7 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         // still in flight would wait for that load).
         static_assert(kAhead == 2, "the stage loop below alternates two register slots");
         uint4 rq0[2], rq1[2];
-        __half2 sq0[4], sq1[4];
+        __half sq0[kScales], sq1[kScales];
         load_next(rq0, sq0);
         load_next(rq1, sq1);
         for (int i = grp; i < nst; i += 2 * DQ) {
@@ -535,11 +532,11 @@ struct Variant {
     int nominal_per_sm;  // the residency the variant is sized for (used when no device is present)
     int tmem_cols;       // TMEM columns each resident CTA allocates
     int smem;
-    const void* fn;
-    int (*launch)(const CUtensorMap&, const Params&, dim3, int, int, cudaStream_t);
+    const void* fn[2];  // [0]: G a multiple of 64 (one scale per stage), [1]: any G
+    int (*launch[2])(const CUtensorMap&, const Params&, dim3, int, int, cudaStream_t);
 };
 
-template <int BN, int LS, int TC, int MINB, int DQ>
+template <int BN, int LS, int TC, int MINB, int DQ, bool OG>
 int launch_variant(const CUtensorMap& map, const Params& p, dim3 grid, int cluster_x, int smem, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -560,15 +557,20 @@ int launch_variant(const CUtensorMap& map, const Params& p, dim3 grid, int clust
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, w4a16_gemm_kernel<BN, LS, TC, MINB, DQ>, map, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, w4a16_gemm_kernel<BN, LS, TC, MINB, DQ, OG>, map, p);
     return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
 template <int BN, int LS, int TC, int MINB, int DQ>
 Variant make_variant() {
-    return Variant{BN, threads_for(DQ), MINB, TC, Layout<BN, LS, TC>::kAlloc,
-                   reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB, DQ>),
-                   &launch_variant<BN, LS, TC, MINB, DQ>};
+    return Variant{BN,
+                   threads_for(DQ),
+                   MINB,
+                   TC,
+                   Layout<BN, LS, TC>::kAlloc,
+                   {reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB, DQ, true>),
+                    reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB, DQ, false>)},
+                   {&launch_variant<BN, LS, TC, MINB, DQ, true>, &launch_variant<BN, LS, TC, MINB, DQ, false>}};
 }
 
 // Token tiles and their pipeline depths: small tiles keep two CTAs per SM; the
@@ -604,24 +606,28 @@ int prepare_device(DeviceState** out) {
     if (!st.ready) {
         for (int i = 0; i < 5; ++i) {
             const Variant& v = kVariants[i];
-            if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess ||
-                cudaFuncSetAttribute(v.fn, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                     cudaSharedmemCarveoutMaxShared) != cudaSuccess)
-                return W4A16_ERR_CUDA;
-            // Residency from the SM's limits (shared memory with its per-block
-            // reservation, registers per warp, threads, TMEM columns).
-            cudaFuncAttributes fa;
-            if (cudaFuncGetAttributes(&fa, v.fn) != cudaSuccess) return W4A16_ERR_CUDA;
-            int smem_sm = 0, resv = 0, regs_sm = 0, threads_sm = 0;
-            cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-            cudaDeviceGetAttribute(&resv, cudaDevAttrReservedSharedMemoryPerBlock, dev);
-            cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
-            cudaDeviceGetAttribute(&threads_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
-            const int per_warp_regs = ((fa.numRegs * 32 + 255) / 256) * 256;
-            int n = smem_sm / (v.smem + static_cast<int>(fa.sharedSizeBytes) + resv);
-            n = std::min(n, regs_sm / (per_warp_regs * (v.threads / 32)));
-            n = std::min(n, threads_sm / v.threads);
-            n = std::min(n, 512 / v.tmem_cols);  // every resident CTA holds its TMEM columns
+            int n = 1 << 30;
+            for (const void* fn : v.fn) {
+                if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess ||
+                    cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+                    return W4A16_ERR_CUDA;
+                // Residency from the SM's limits (shared memory with its per-block
+                // reservation, registers per warp, threads, TMEM columns); the
+                // smaller of the variant's two forms.
+                cudaFuncAttributes fa;
+                if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return W4A16_ERR_CUDA;
+                int smem_sm = 0, resv = 0, regs_sm = 0, threads_sm = 0;
+                cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+                cudaDeviceGetAttribute(&resv, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+                cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+                cudaDeviceGetAttribute(&threads_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
+                const int per_warp_regs = ((fa.numRegs * 32 + 255) / 256) * 256;
+                n = std::min(n, smem_sm / (v.smem + static_cast<int>(fa.sharedSizeBytes) + resv));
+                n = std::min(n, regs_sm / (per_warp_regs * (v.threads / 32)));
+                n = std::min(n, threads_sm / v.threads);
+                n = std::min(n, 512 / v.tmem_cols);  // every resident CTA holds its TMEM columns
+            }
             if (n < 1) return W4A16_ERR_UNSUPPORTED;
             st.ctas_per_sm[i] = n;
         }
@@ -880,7 +886,7 @@ extern "C" int w4a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt_dev, const 
     rc = make_act_map(&map, A_dev, M, K, plan.bn);
     if (rc) return rc;
     const Variant& v = variant_for(plan.bn);
-    return v.launch(map, p, plan.grid, plan.splits, v.smem, static_cast<cudaStream_t>(stream));
+    return v.launch[(G % kTileK) ? 1 : 0](map, p, plan.grid, plan.splits, v.smem, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const* Wt, const w4a16_half* const* S,
@@ -929,7 +935,7 @@ extern "C" int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const*
     rc = make_act_map(&map, A_dev, total_rows, K, plan.bn);
     if (rc) return rc;
     const Variant& v = variant_for(plan.bn);
-    return v.launch(map, p, plan.grid, 1, v.smem, static_cast<cudaStream_t>(stream));
+    return v.launch[(G % kTileK) ? 1 : 0](map, p, plan.grid, 1, v.smem, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int w4a16_device_status(int clear) {
