@@ -239,6 +239,65 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         tma_load_2d(smem + L::kAct + s * L::kActBytes, &tmA, (kb + i) * kTileK, m0, &full[s]);
     };
 
+    // ---- dequantisation threads' state (warps 2..). Their first look-ahead
+    // loads go out before the barrier and TMEM setup below, so that the
+    // first stage's memory latency overlaps it.
+    const int dw = warp - 2;
+    const int grp = dw >> 2;          // dequantisation group: stages grp, grp + DQ, ...
+    const int quad = warp & 3;        // TMEM lane quadrant this warp may access
+    const int j = quad * 32 + lane;   // weight column inside the tile = TMEM lane
+    const int n = nt * kTileN + j;
+    const bool col_ok = n < p.N;
+    const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
+    // Codes and scales of this thread's stages (i = grp, grp + DQ, ...) are
+    // loaded kAhead of its stages ahead into registers: the two 16-byte
+    // halves (k 0..31 and 32..63) of the column's stage and its scales (one
+    // when G is a multiple of 64, else one per 8-deep word). Loaded values
+    // are left exactly as loaded until the stage is decoded: any instruction
+    // that reads a register whose load is in flight waits for that load.
+    // kk is the first k of the next stage to load, gk = floor(kk / G).
+    // (A padded column past N reads column 0's scales; its codes are 0.)
+    const uint8_t* wcol = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes + j * 16;
+    const __half* scol = p.sc[expert] + (col_ok ? n : 0);
+    int li = grp;
+    int kk = (kb + grp) * kTileK;
+    int gk = kk / p.G;
+    auto load_next = [&](uint4 (&r)[2], __half (&sv)[kScales]) {
+        if (li < nst) {
+            const uint8_t* src = wcol + static_cast<int64_t>(kb + li) * kRawBytes;
+            r[0] = ld_nc_v4(src);
+            r[1] = ld_nc_v4(src + kRawBytes / 2);
+            if constexpr (OG) {
+                sv[0] = __ldg(scol + static_cast<int64_t>(min(gk, p.ngroups - 1)) * p.N);
+            } else {
+                const int rem = kk - gk * p.G;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    int g = gk, r2 = rem + 8 * q;
+                    while (r2 >= p.G) {
+                        r2 -= p.G;
+                        ++g;
+                    }
+                    sv[q] = __ldg(scol + static_cast<int64_t>(min(g, p.ngroups - 1)) * p.N);
+                }
+            }
+        } else {
+            r[0] = r[1] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int q = 0; q < kScales; ++q) sv[q] = __float2half(0.f);
+        }
+        li += DQ;
+        kk += kTileK * DQ;
+        while ((gk + 1) * p.G <= kk) ++gk;
+    };
+    uint4 rq0[2], rq1[2];
+    __half sq0[kScales], sq1[kScales];
+    if (warp >= 2) {
+        if (!p.prefetch) grid_dependency_wait();  // weights and scales may come from the previous kernel
+        load_next(rq0, sq0);
+        load_next(rq1, sq1);
+    }
+
     if (threadIdx.x == 0) {
         for (int s = 0; s < LS; ++s) {
             mbar_init(&full[s], 1);
@@ -270,9 +329,13 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             // The int4 tile of a stage is one contiguous 4 KB block: pull it into
             // L2 kPrefetchStages ahead, so that the dequantising threads' own
             // loads (issued only kAhead of their stages ahead) find it there.
+            // (The ring's first LS activation tiles go out before the prefetches.)
             const uint8_t* wtile = p.wt[expert] + (static_cast<int64_t>(nt) * p.KT + kb) * kRawBytes;
-            for (int i = 0; i < min(nst, kPrefetchStages); ++i) bulk_prefetch_l2(wtile + static_cast<int64_t>(i) * kRawBytes, kRawBytes);
-            int issued = 0;
+            const int first = min(nst, LS);
+            for (int i = 0; i < first; ++i) issue_act(i);
+            for (int i = 0; i < min(nst, kPrefetchStages + first); ++i)
+                bulk_prefetch_l2(wtile + static_cast<int64_t>(i) * kRawBytes, kRawBytes);
+            int issued = first;
             for (; issued < nst; ++issued) {
                 const int i = issued;
                 if (i >= LS && !wait_phase(&done[i % LS], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
@@ -317,55 +380,6 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         __syncwarp();
     } else {
         // ------------------------------------------------------ dequant + epilogue
-        const int dw = warp - 2;
-        const int grp = dw >> 2;          // dequantisation group: stages grp, grp + DQ, ...
-        const int quad = warp & 3;        // TMEM lane quadrant this warp may access
-        const int j = quad * 32 + lane;   // weight column inside the tile = TMEM lane
-        const int n = nt * kTileN + j;
-        const bool col_ok = n < p.N;
-        const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
-        // Codes and scales of this thread's stages (i = grp, grp + DQ, ...) are
-        // loaded kAhead of its stages ahead into registers: the two 16-byte
-        // halves (k 0..31 and 32..63) of the column's stage and its scales (one
-        // when G is a multiple of 64, else one per 8-deep word). Loaded values
-        // are left exactly as loaded until the stage is decoded: any instruction
-        // that reads a register whose load is in flight waits for that load.
-        // kk is the first k of the next stage to load, gk = floor(kk / G).
-        // (A padded column past N reads column 0's scales; its codes are 0.)
-        const uint8_t* wcol = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes + j * 16;
-        const __half* scol = p.sc[expert] + (col_ok ? n : 0);
-        int li = grp;
-        int kk = (kb + grp) * kTileK;
-        int gk = kk / p.G;
-        auto load_next = [&](uint4 (&r)[2], __half (&sv)[kScales]) {
-            if (li < nst) {
-                const uint8_t* src = wcol + static_cast<int64_t>(kb + li) * kRawBytes;
-                r[0] = ld_nc_v4(src);
-                r[1] = ld_nc_v4(src + kRawBytes / 2);
-                if constexpr (OG) {
-                    sv[0] = __ldg(scol + static_cast<int64_t>(min(gk, p.ngroups - 1)) * p.N);
-                } else {
-                    const int rem = kk - gk * p.G;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        int g = gk, r2 = rem + 8 * q;
-                        while (r2 >= p.G) {
-                            r2 -= p.G;
-                            ++g;
-                        }
-                        sv[q] = __ldg(scol + static_cast<int64_t>(min(g, p.ngroups - 1)) * p.N);
-                    }
-                }
-            } else {
-                r[0] = r[1] = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                for (int q = 0; q < kScales; ++q) sv[q] = __float2half(0.f);
-            }
-            li += DQ;
-            kk += kTileK * DQ;
-            while ((gk + 1) * p.G <= kk) ++gk;
-        };
-        if (!p.prefetch) grid_dependency_wait();  // weights and scales may come from the previous kernel
         // One stage: decode the codes and scales held in (r, sv), refill them
         // with the thread's stage kAhead of its stages later, store the fp16
         // weights into the stage's TMEM slot and arrive. False when aborting.
@@ -403,10 +417,6 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         // the registers they were loaded into (moving a register whose load is
         // still in flight would wait for that load).
         static_assert(kAhead == 2, "the stage loop below alternates two register slots");
-        uint4 rq0[2], rq1[2];
-        __half sq0[kScales], sq1[kScales];
-        load_next(rq0, sq0);
-        load_next(rq1, sq1);
         for (int i = grp; i < nst; i += 2 * DQ) {
             if (!stage(i, rq0, sq0)) break;
             if (i + DQ < nst && !stage(i + DQ, rq1, sq1)) break;
@@ -425,14 +435,23 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             // Stage the fp16 tile, row-major [token][128 columns], in the idle
             // activation ring (every copy into it was consumed by a completed
             // MMA), so that the global stores below are whole 16-byte vectors.
+            // Two 16-token chunks per TMEM wait.
             if (have_acc) {
                 __half* stile = reinterpret_cast<__half*>(smem + L::kAct);
-                for (int c = grp; c < n_mma / 16; c += DQ) {
-                    uint32_t v[16];
+                const int nch = n_mma / 16;
+                for (int c = grp; c < nch; c += 2 * DQ) {
+                    const bool two = c + DQ < nch;
+                    uint32_t v[16], w[16];
                     tmem_ld_32x32b_x16(tmem_acc + tlane + c * 16, v);
+                    if (two) tmem_ld_32x32b_x16(tmem_acc + tlane + (c + DQ) * 16, w);
                     tmem_ld_wait();
 #pragma unroll
                     for (int t = 0; t < 16; ++t) stile[(c * 16 + t) * kTileN + j] = __float2half_rn(__uint_as_float(v[t]));
+                    if (two) {
+#pragma unroll
+                        for (int t = 0; t < 16; ++t)
+                            stile[((c + DQ) * 16 + t) * kTileN + j] = __float2half_rn(__uint_as_float(w[t]));
+                    }
                 }
             }
         } else {
