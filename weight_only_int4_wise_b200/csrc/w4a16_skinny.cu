@@ -277,9 +277,13 @@ int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan) {
     const int mt = M <= 8 ? 1 : 2;
     int sms = sm_count();
     if (sms <= 0) sms = 148;
-    // Up to two CTAs per SM in a single wave (a second wave of clusters would
-    // double the time), never more than the cluster limit or the K blocks.
-    int64_t splits = (2 * sms) / NT;
+    // One wave (a second wave of clusters would double the time), never more
+    // than the cluster limit or the K blocks. One token tile: one CTA per SM,
+    // so that every SM does the same share (with two per SM on some SMs and
+    // one on others, the clusters wait for the doubly loaded ones: measured
+    // 6.7 against 7.6 us at K = N = 4096). Two token tiles, with twice the
+    // MMA work per weight, spread over up to two CTAs per SM.
+    int64_t splits = (mt == 1 ? sms : 2 * sms) / NT;
     if (splits > 8) splits = 8;
     if (splits > KB) splits = KB;
     if (splits < 1) splits = 1;
