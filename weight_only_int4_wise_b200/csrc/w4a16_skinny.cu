@@ -142,9 +142,12 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
     }
     __syncthreads();  // staged activations are visible; scales are waited for with block 0
 
-    float acc[MT][4];
+    float acc[MT][4], acc2[MT][4];  // (acc2: the odd-step chain when groups are finer than a block)
 #pragma unroll
-    for (int j = 0; j < MT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    for (int j = 0; j < MT; ++j) {
+        acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+        acc2[j][0] = acc2[j][1] = acc2[j][2] = acc2[j][3] = 0.f;
+    }
     uint32_t arow[MT];
 #pragma unroll
     for (int j = 0; j < MT; ++j) arow[j] = smem_addr(act + (8 * j + g) * p.act_stride + 32 * t);
@@ -160,9 +163,11 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
         const uint32_t wa_w[4] = {wa.x, wa.y, wa.z, wa.w};
         const uint32_t wb_w[4] = {wb.x, wb.y, wb.z, wb.w};
         if (p.post_scale) {
-            // One group covers the whole block: one MMA chain over the exact codes,
-            // started from a zero accumulator, then one scaled add per element.
-            float part[MT][4];
+            // One group covers the whole block: MMA chains over the exact codes,
+            // started from zero accumulators, then one scaled add per element.
+            // Two chains (even and odd 16-deep steps) halve the dependent MMA
+            // latency; their sum is taken in a fixed order.
+            float part[2][MT][4];
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
                 const uint4 qa = decode_word(wa_w[w]);
@@ -174,10 +179,10 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
 #pragma unroll
                     for (int j = 0; j < MT; ++j) {
                         const uint2 bfr = lds64(arow[j] + kb2 + 8 * st);
-                        if (st == 0)
-                            mma_m16n8k16_zc(part[j], afr, bfr.x, bfr.y);
+                        if (w == 0)
+                            mma_m16n8k16_zc(part[u][j], afr, bfr.x, bfr.y);
                         else
-                            mma_m16n8k16(part[j], afr, bfr.x, bfr.y);
+                            mma_m16n8k16(part[u][j], afr, bfr.x, bfr.y);
                     }
                 }
             }
@@ -186,10 +191,10 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
             const float sb = __half2float(scl[gr * 128 + ja + 8]);
 #pragma unroll
             for (int j = 0; j < MT; ++j) {
-                acc[j][0] = fmaf(part[j][0], sa, acc[j][0]);
-                acc[j][1] = fmaf(part[j][1], sa, acc[j][1]);
-                acc[j][2] = fmaf(part[j][2], sb, acc[j][2]);
-                acc[j][3] = fmaf(part[j][3], sb, acc[j][3]);
+                acc[j][0] = fmaf(part[0][j][0] + part[1][j][0], sa, acc[j][0]);
+                acc[j][1] = fmaf(part[0][j][1] + part[1][j][1], sa, acc[j][1]);
+                acc[j][2] = fmaf(part[0][j][2] + part[1][j][2], sb, acc[j][2]);
+                acc[j][3] = fmaf(part[0][j][3] + part[1][j][3], sb, acc[j][3]);
             }
         } else {
             // Groups finer than the block: scale each decoded word (rounded to fp16).
@@ -207,7 +212,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
 #pragma unroll
                     for (int j = 0; j < MT; ++j) {
                         const uint2 bfr = lds64(arow[j] + kb2 + 8 * st);
-                        mma_m16n8k16(acc[j], afr, bfr.x, bfr.y);
+                        mma_m16n8k16(u ? acc2[j] : acc[j], afr, bfr.x, bfr.y);  // two chains
                     }
                 }
             }
@@ -215,6 +220,13 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
         issue_block(i + kDepth);  // this thread's slot for block i is consumed (values decoded above)
     }
     cp_async_wait<0>();
+    if (!p.post_scale) {
+#pragma unroll
+        for (int j = 0; j < MT; ++j) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[j][e] += acc2[j][e];
+        }
+    }
 
     const int na = nt * 128 + ja;
     if (S == 1) {
