@@ -356,22 +356,33 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             // the dequantised weights and, through each group's first warp, the
             // landed activation tiles. (Each wait costs the single issuing thread
             // about as long as an MMA, so it is paid once per eight MMAs.)
+            // (The ring is unrolled: each slot's descriptors are constants.)
             const uint64_t bdesc0 = smem_desc_k_sw128(smem_addr(smem + L::kAct));
-            for (int i = 0; i < nst; i += 2) {
-                const int q = i >> 1;
-                if (!wait_phase(&afull[q % (LS / 2)], static_cast<uint32_t>(q / (LS / 2)) & 1u, abort_flag)) break;
-                tc_fence_after_sync();
+            bool stop = false;
+            for (int base = 0; base < nst && !stop; base += LS) {
+                const uint32_t par = static_cast<uint32_t>(base / LS) & 1u;
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    if (i + t < nst) {
-                        const int s = (i + t) % LS;
-                        const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((s * L::kActBytes) >> 4);
-                        const uint32_t a0 = tmem_ring + s * kSlotCols;
-                        mma_f16_ts(tmem_acc, a0, bdesc, idesc, (i + t) > 0 ? 1u : 0u);
-                        mma_f16_ts(tmem_acc, a0 + 8, bdesc + 2, idesc, 1u);
-                        mma_f16_ts(tmem_acc, a0 + 16, bdesc + 4, idesc, 1u);
-                        mma_f16_ts(tmem_acc, a0 + 24, bdesc + 6, idesc, 1u);
-                        mma_commit(&done[s]);
+                for (int qq = 0; qq < LS / 2; ++qq) {
+                    const int i = base + 2 * qq;
+                    if (i >= nst) break;
+                    if (!wait_phase(&afull[qq], par, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        if (i + t < nst) {
+                            constexpr uint64_t kStep = static_cast<uint64_t>(L::kActBytes >> 4);
+                            const int s = 2 * qq + t;
+                            const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s) * kStep;
+                            const uint32_t a0 = tmem_ring + static_cast<uint32_t>(s * kSlotCols);
+                            mma_f16_ts(tmem_acc, a0, bdesc, idesc, (i + t) > 0 ? 1u : 0u);
+                            mma_f16_ts(tmem_acc, a0 + 8, bdesc + 2, idesc, 1u);
+                            mma_f16_ts(tmem_acc, a0 + 16, bdesc + 4, idesc, 1u);
+                            mma_f16_ts(tmem_acc, a0 + 24, bdesc + 6, idesc, 1u);
+                            mma_commit(&done[s]);
+                        }
                     }
                 }
             }
