@@ -94,10 +94,20 @@ def _addr(x) -> Optional[int]:
     return x.data_ptr()
 
 
+def _current_stream(device_index: Optional[int] = None) -> int:
+    """Raw handle of torch's current stream (the cheap accessor when torch has it)."""
+    import torch
+    if device_index is None:
+        device_index = torch.cuda.current_device()
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None:
+        return raw(device_index)
+    return torch.cuda.current_stream(device_index).cuda_stream
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
-        import torch
-        return torch.cuda.current_stream().cuda_stream
+        return _current_stream()
     if isinstance(stream, int):
         return stream
     return stream.cuda_stream
@@ -209,12 +219,20 @@ def prepare_weights(q, stream=None):
 def gemm(A, wt, S, N: int, G: int, out=None, stream=None):
     """C [M, N] fp16 = A [M, K] fp16 x dequant(tiled weights, scales S [ceil(K/G), N])."""
     import torch
-    _require_cuda(A, wt, S)
+    if not (A.is_cuda and wt.is_cuda and S.is_cuda):
+        raise ValueError("all tensors must live on a CUDA device")
     if A.dtype != torch.float16 or S.dtype != torch.float16:
         raise TypeError("A and S must be float16")
     M, K = A.shape
+    if not A.is_contiguous():
+        A = A.contiguous()
+    if not S.is_contiguous():
+        S = S.contiguous()
     C = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=A.device)
-    _check(w4a16_gemm(A.contiguous(), wt, S.contiguous(), C, M, N, K, G, stream), "w4a16_gemm")
+    st = _current_stream(A.device.index) if stream is None else _stream(stream)
+    rc = (_lib or load()).w4a16_gemm(A.data_ptr(), wt.data_ptr(), S.data_ptr(), C.data_ptr(), M, N, K, G, st)
+    if rc != OK:
+        raise W4A16Error(rc, "w4a16_gemm")
     return C
 
 

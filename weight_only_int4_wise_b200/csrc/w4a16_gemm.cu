@@ -779,26 +779,25 @@ void fill_info(const Plan& plan, w4a16_launch_info* info) {
 }  // namespace
 
 int check_device() {
-    static int cached[64];
-    static bool known[64];
-    static std::mutex mu;
+    // per device: 0 unknown, 1 supported, 2 not (cached: this runs on every call)
+    static std::atomic<int> state[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
         return W4A16_ERR_UNSUPPORTED;
     }
     if (dev < 0 || dev >= 64) return W4A16_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!known[dev]) {
+    int st = state[dev].load(std::memory_order_acquire);
+    if (st == 0) {
         int major = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
             cudaGetLastError();
             return W4A16_ERR_UNSUPPORTED;
         }
-        cached[dev] = (major == 10) ? W4A16_OK : W4A16_ERR_UNSUPPORTED;
-        known[dev] = true;
+        st = (major == 10) ? 1 : 2;
+        state[dev].store(st, std::memory_order_release);
     }
-    return cached[dev];
+    return st == 1 ? W4A16_OK : W4A16_ERR_UNSUPPORTED;
 }
 
 namespace {
@@ -808,9 +807,13 @@ std::atomic<int> g_static_weights{0};
 bool static_weights_enabled() { return g_static_weights.load(std::memory_order_relaxed) != 0; }
 
 int sm_count() {
+    static std::atomic<int> cached[64];
     int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    n = cached[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 

@@ -322,11 +322,18 @@ int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan) {
         ++splits;
     }
     if (NT > 65535) return W4A16_ERR_UNSUPPORTED;
-    // floor(k / G) as a multiply-shift, checked exhaustively over the padded K range.
+    // floor(k / G) as a multiply-shift over the padded K range. With
+    // magic = (2^32 + e) / G, 0 <= e < G, k * magic / 2^32 = k / G + k * e / (G * 2^32),
+    // which floors to floor(k / G) whenever k * e < 2^32 (the fractional part of
+    // k / G is at most (G - 1) / G). Otherwise every k is checked.
     const uint64_t magic = ((uint64_t(1) << 32) + static_cast<uint64_t>(G) - 1) / static_cast<uint64_t>(G);
     if (magic > 0xFFFFFFFFull) return W4A16_ERR_UNSUPPORTED;
-    for (int64_t k = 0; k < KB * kBlockK; k += 8)
-        if (static_cast<int64_t>((static_cast<uint64_t>(k) * magic) >> 32) != k / G) return W4A16_ERR_UNSUPPORTED;
+    const uint64_t e = magic * static_cast<uint64_t>(G) - (uint64_t(1) << 32);
+    const uint64_t kend = static_cast<uint64_t>(KB * kBlockK);
+    if (e != 0 && kend > ((uint64_t(1) << 32) - 1) / e) {
+        for (int64_t k = 0; k < KB * kBlockK; k += 8)
+            if (static_cast<int64_t>((static_cast<uint64_t>(k) * magic) >> 32) != k / G) return W4A16_ERR_UNSUPPORTED;
+    }
     plan->g_magic = static_cast<uint32_t>(magic);
     plan->post_scale = (G % kBlockK) == 0 ? 1 : 0;
     return W4A16_OK;
