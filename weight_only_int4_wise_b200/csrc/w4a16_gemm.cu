@@ -6,24 +6,29 @@
 // groupSize G). The grouped-expert entry point applies it per expert segment
 // of gathered rows (Int4MoePlugin page, constructor parameters).
 //
-// One kernel template serves decode (M = 1..16), skinny, prefill and
-// grouped-expert shapes. It computes the transposed product
+// One kernel template serves M > 16 (decode-sized M runs on the skinny
+// kernel) and the grouped-expert form. It computes the transposed product
 //     D[n, m] = sum_k W[k, n] * A[m, k]
 // on the 5th-generation tensor core: each CTA owns 128 weight columns (the MMA
 // M extent, one TMEM lane per column) and a tile of BN activation rows (the
 // MMA N extent, 16..256), so that small token counts cost no padding of the
 // weight side. Warp roles inside a CTA (320 or 576 threads):
 //   warp 0      producer: per 64-deep K stage, one TMA tile load of the
-//               activations (128-byte swizzle, zero fill past M and K).
+//               activations (128-byte swizzle, zero fill past M and K) into a
+//               ring of stages, and an L2 prefetch of the column tile's int4
+//               stages well ahead of use.
 //   warp 1      TMEM allocation and the single MMA-issuing thread
-//               (tcgen05.mma kind::f16, fp32 accumulator in TMEM).
-//   warps 2..   dequantisation, in one or two groups of 8 warps (group g takes
-//               stages g, g + groups, ...): each thread loads 32 int4 codes of
-//               one column (16 bytes of the tiled layout) and their scales
-//               straight into registers two of its stages ahead, turns them
-//               into fp16 (magic-exponent decode, times the group scale) and
-//               stores them into the stage's tensor-memory slot; then the
-//               epilogue (tcgen05.ld -> fp16 -> global).
+//               (tcgen05.mma kind::f16, A = weights from TMEM, B = activations
+//               from shared memory, fp32 accumulator in TMEM); it waits on one
+//               barrier per pair of stages.
+//   warps 2..   dequantisation, in groups of four warps (one per TMEM lane
+//               quadrant; group g takes stages g, g + groups, ...): each thread
+//               loads its column's 64 int4 codes of a stage (two 16-byte halves
+//               of the tiled layout) and their scale straight into registers,
+//               two of its stages ahead, turns them into fp16 (magic-exponent
+//               decode, times the group scale) and stores them into the
+//               stage's tensor-memory slot; then the epilogue (tcgen05.ld ->
+//               fp16 tile in shared memory -> 16-byte row stores).
 // Small-M shapes split K across up to 8 CTAs of one thread-block cluster; the
 // fp32 partial tiles are summed in rank order through distributed shared
 // memory (deterministic, no global workspace).

@@ -14,7 +14,8 @@
 //     previous kernel in the stream has finished (programmatic dependent
 //     launch lets the weight copies start before that);
 //   - K is split over up to 8 CTAs of a thread-block cluster whose fp32 partial
-//     tiles are summed in rank order in the owning CTA's shared memory.
+//     tiles are summed in rank order in the owning CTA's shared memory (one
+//     token tile: sized for one CTA per SM; two token tiles: up to two).
 //
 // Fragment mapping. Inside a 16-deep MMA step the k order is free as long as
 // both operands use it. Thread (g = lane/4, t = lane%4) holds, for output
