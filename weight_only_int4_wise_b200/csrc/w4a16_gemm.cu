@@ -616,19 +616,20 @@ Variant make_variant() {
 // slower on the prefill and grouped-expert shapes.
 // <token tile, ring stages, TMEM columns, CTAs per SM, dequantisation groups>
 const Variant kVariants[] = {
-    make_variant<16, 6, 256, 2, 2>(), make_variant<32, 6, 256, 2, 2>(), make_variant<64, 6, 256, 2, 2>(),
-    make_variant<128, 4, 256, 2, 2>(), make_variant<256, 6, 512, 1, 4>(),
+    make_variant<16, 6, 256, 2, 2>(),  make_variant<32, 6, 256, 2, 2>(),  make_variant<64, 6, 256, 2, 2>(),
+    make_variant<128, 4, 256, 2, 2>(), make_variant<192, 8, 512, 1, 4>(), make_variant<256, 6, 512, 1, 4>(),
 };
+constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
 const Variant& variant_for(int bn) {
     for (const Variant& v : kVariants)
         if (v.bn == bn) return v;
-    return kVariants[4];
+    return kVariants[kNumVariants - 1];
 }
 
 struct DeviceState {
     bool ready = false;
-    int ctas_per_sm[5] = {0, 0, 0, 0, 0};
+    int ctas_per_sm[kNumVariants] = {};
 };
 
 int prepare_device(DeviceState** out) {
@@ -639,7 +640,7 @@ int prepare_device(DeviceState** out) {
     std::lock_guard<std::mutex> lock(mu);
     DeviceState& st = states[dev];
     if (!st.ready) {
-        for (int i = 0; i < 5; ++i) {
+        for (int i = 0; i < kNumVariants; ++i) {
             const Variant& v = kVariants[i];
             int n = 1 << 30;
             for (const void* fn : v.fn) {
@@ -673,9 +674,9 @@ int prepare_device(DeviceState** out) {
 }
 
 int variant_index(int bn) {
-    for (int i = 0; i < 5; ++i)
+    for (int i = 0; i < kNumVariants; ++i)
         if (kVariants[i].bn == bn) return i;
-    return 4;
+    return kNumVariants - 1;
 }
 
 int token_tile_for(int64_t rows_per_tile) {
@@ -683,6 +684,7 @@ int token_tile_for(int64_t rows_per_tile) {
     if (rows_per_tile <= 32) return 32;
     if (rows_per_tile <= 64) return 64;
     if (rows_per_tile <= 128) return 128;
+    if (rows_per_tile <= 192) return 192;
     return 256;
 }
 
