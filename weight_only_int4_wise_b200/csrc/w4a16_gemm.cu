@@ -859,7 +859,7 @@ extern "C" int w4a16_gemm_launch_info(int64_t M, int64_t N, int64_t K, int64_t G
         info->grid_x = sk.grid_x;
         info->grid_y = sk.grid_y;
         info->grid_z = 1;
-        info->threads_per_cta = 256;
+        info->threads_per_cta = sk.threads;
         info->smem_bytes = sk.smem;
         info->ctas_per_sm = (228 * 1024) / (sk.smem + 1024) < 2 ? (228 * 1024) / (sk.smem + 1024) : 2;
         return W4A16_OK;

@@ -24,8 +24,9 @@ constexpr int kSkinnyMaxM = 16;
 
 struct SkinnyPlan {
     int mt;             // token tiles of 8 rows (1 or 2)
+    int threads;        // threads per CTA (256 per K half)
     int splits;         // CTAs along K in one cluster
-    int depth;          // 128-deep K blocks in flight per thread (4 or 8)
+    int depth;          // 128-deep K blocks in flight per thread (2 to 8)
     int grid_x, grid_y;
     int act_stride;     // staged activation row, in halves
     int scale_rows;     // staged scale rows

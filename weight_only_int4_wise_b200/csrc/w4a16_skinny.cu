@@ -39,7 +39,7 @@ namespace w4a16 {
 namespace {
 
 constexpr int kSkWarps = 8;                       // 8 warps x 16 columns = one 128-column weight tile
-constexpr int kSkThreads = kSkWarps * 32;
+constexpr int kSkThreads = kSkWarps * 32;         // threads of one K half
 constexpr int kBlockK = 128;
 constexpr int kSlotBytes = 32;                    // per thread and block: two 16-byte chunks
 
@@ -63,10 +63,16 @@ struct SkinnyParams {
     int32_t prefetch;         // weights/scales may be read before the previous kernel finishes
 };
 
-template <int MT, int kDepth>
-__global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __grid_constant__ SkinnyParams p) {
+// KH = 2 runs two sets of 8 warps over the same 128 columns, the first taking
+// the even 128-deep blocks of the CTA's K range and the second the odd ones, and
+// adds the two partial tiles in shared memory (first + second) after the loop.
+template <int MT, int kDepth, int KH>
+__global__ void __launch_bounds__(KH * kSkThreads, 2)
+    w4a16_skinny_kernel(const __grid_constant__ SkinnyParams p) {
     extern __shared__ __align__(1024) uint8_t sm[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kThreads = KH * kSkThreads;
+    const int warp = (threadIdx.x >> 5) & (kSkWarps - 1), lane = threadIdx.x & 31;
+    const int kh = static_cast<int>(threadIdx.x) / kSkThreads;  // K half: blocks i with i % KH == kh
     const int g = lane >> 2, t = lane & 3;
     const int split = blockIdx.x, nt = blockIdx.y;
     const int b0 = static_cast<int>((static_cast<int64_t>(split) * p.KB) / p.splits);
@@ -81,7 +87,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
     __half* act = reinterpret_cast<__half*>(sm);                          // [MP][act_stride]
     __half* scl = act + MP * p.act_stride;                                // [scale_rows][128]
     uint8_t* ring = reinterpret_cast<uint8_t*>(scl + p.scale_rows * 128); // [kDepth][2][threads][16 B]
-    float* red = reinterpret_cast<float*>(ring + kDepth * kSkThreads * kSlotBytes);  // [S][MP][cwm] partials
+    float* red = reinterpret_cast<float*>(ring + kDepth * kThreads * kSlotBytes);  // [S][MP][cwm] partials
 
     const int g_lo = kr0 / p.G;
     const int g_hi = min(p.ngroups - 1, (kr0 + krange - 1) / p.G);
@@ -92,20 +98,22 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
     // half t%2. A missing second tile at an odd end of K reads as zeros.
     const uint8_t* wsrc = p.wt + (static_cast<int64_t>(nt) * p.KT + 2 * b0 + (t >> 1)) * 4096 + (t & 1) * 2048 + ja * 16;
     const int kt_last_ok = p.KT - 1 - (t >> 1);
-    uint8_t* myslot = ring + threadIdx.x * 16;  // chunk of column ja; column ja + 8's is kSkThreads * 16 further
-    auto issue_block = [&](int i) {
+    uint8_t* myslot = ring + threadIdx.x * 16;  // chunk of column ja; column ja + 8's is kThreads * 16 further
+    // Local block li of this half is block i = li * KH + kh, in slot li % kDepth.
+    auto issue_block = [&](int li) {
+        const int i = li * KH + kh;
         if (i < nb) {
             const bool ok = 2 * (b0 + i) <= kt_last_ok;
             const uint8_t* src = wsrc + static_cast<int64_t>(i) * 8192;
-            uint8_t* dst = myslot + (i % kDepth) * kSkThreads * kSlotBytes;
+            uint8_t* dst = myslot + (li % kDepth) * kThreads * kSlotBytes;
             cp_async16(dst, ok ? src : p.wt, ok ? 16u : 0u);
-            cp_async16(dst + kSkThreads * 16, ok ? src + 128 : p.wt, ok ? 16u : 0u);
+            cp_async16(dst + kThreads * 16, ok ? src + 128 : p.wt, ok ? 16u : 0u);
         }
         cp_async_commit();  // one group per block, empty past the end, so the counts stay uniform
     };
     auto issue_scales = [&]() {
         const int ncols = min(128, p.N - nt * 128);
-        for (int idx = threadIdx.x; idx < nrows * 16; idx += kSkThreads) {
+        for (int idx = threadIdx.x; idx < nrows * 16; idx += kThreads) {
             const int r = idx >> 4, c = idx & 15;
             const bool ok = c * 8 < ncols;
             cp_async16(scl + r * 128 + c * 8,
@@ -133,7 +141,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
     }
     {
         const int cpr = krange / 8;  // 16-byte chunks per activation row
-        for (int idx = threadIdx.x; idx < MP * cpr; idx += kSkThreads) {
+        for (int idx = threadIdx.x; idx < MP * cpr; idx += kThreads) {
             const int r = idx / cpr, c = idx - r * cpr;
             const int k = kr0 + c * 8;
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -141,7 +149,8 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
             *reinterpret_cast<uint4*>(act + r * p.act_stride + c * 8) = v;
         }
     }
-    __syncthreads();  // staged activations are visible; scales are waited for with block 0
+    cp_async_wait<kDepth - 1>();  // the scale rows (and this thread's first block) have landed
+    __syncthreads();              // staged activations and scale rows are visible to all threads
 
     float acc[MT][4], acc2[MT][4];  // (acc2: the odd-step chain when groups are finer than a block)
 #pragma unroll
@@ -154,12 +163,13 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
     for (int j = 0; j < MT; ++j) arow[j] = smem_addr(act + (8 * j + g) * p.act_stride + 32 * t);
     const uint32_t slot0 = smem_addr(myslot);
 
-    for (int i = 0; i < nb; ++i) {
-        cp_async_wait<kDepth - 1>();  // block i (and the scales) are in this thread's slot
-        if (i == 0) __syncthreads();  // the scale rows were copied by all threads
-        const uint32_t slot = slot0 + (i % kDepth) * kSkThreads * kSlotBytes;
+    const int nbh = (nb - kh + KH - 1) / KH;  // blocks of this half
+    for (int li = 0; li < nbh; ++li) {
+        cp_async_wait<kDepth - 1>();  // local block li is in this thread's slot
+        const int i = li * KH + kh;
+        const uint32_t slot = slot0 + (li % kDepth) * kThreads * kSlotBytes;
         const uint4 wa = lds128(slot);
-        const uint4 wb = lds128(slot + kSkThreads * 16);
+        const uint4 wb = lds128(slot + kThreads * 16);
         const uint32_t kb2 = static_cast<uint32_t>(i * kBlockK * 2);  // block offset in the staged range, bytes
         const uint32_t wa_w[4] = {wa.x, wa.y, wa.z, wa.w};
         const uint32_t wb_w[4] = {wb.x, wb.y, wb.z, wb.w};
@@ -218,7 +228,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
                 }
             }
         }
-        issue_block(i + kDepth);  // this thread's slot for block i is consumed (values decoded above)
+        issue_block(li + kDepth);  // this thread's slot for local block li is consumed (values decoded above)
     }
     cp_async_wait<0>();
     if (!p.post_scale) {
@@ -228,9 +238,29 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
             for (int e = 0; e < 4; ++e) acc[j][e] += acc2[j][e];
         }
     }
+    if (KH == 2) {
+        // The second half's partials go through the (drained) ring; the first half adds them.
+        float* xr = reinterpret_cast<float*>(ring);
+        const int lt = threadIdx.x & (kSkThreads - 1);
+        __syncthreads();  // every thread's copies into the ring have completed
+        if (kh == 1) {
+#pragma unroll
+            for (int j = 0; j < MT; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) xr[(j * 4 + e) * kSkThreads + lt] = acc[j][e];
+        }
+        __syncthreads();
+        if (kh == 0) {
+#pragma unroll
+            for (int j = 0; j < MT; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[j][e] += xr[(j * 4 + e) * kSkThreads + lt];
+        }
+    }
 
     const int na = nt * 128 + ja;
     if (S == 1) {
+        if (kh != 0) return;
 #pragma unroll
         for (int j = 0; j < MT; ++j) {
             const int m0 = 8 * j + 2 * t;
@@ -249,21 +279,24 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
     // [ceil(q*128/S), ceil((q+1)*128/S))), one cluster barrier publishes them,
     // and each owner sums its S slices in rank order.
     const int rank = static_cast<int>(cluster_ctarank());
+    if (kh == 0) {
 #pragma unroll
-    for (int j = 0; j < MT; ++j) {
-        const int m0 = 8 * j + 2 * t;
+        for (int j = 0; j < MT; ++j) {
+            const int m0 = 8 * j + 2 * t;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int m = m0 + (e & 1);
-            const int col = ja + ((e >> 1) << 3);
-            const int q = (col * S) >> 7;          // owner of this column
-            const int cq = (q * 128 + S - 1) / S;  // owner's first column
-            if (m < p.M) st_dsmem_f32(&red[(rank * MP + m) * cwm + (col - cq)], static_cast<uint32_t>(q), acc[j][e]);
+            for (int e = 0; e < 4; ++e) {
+                const int m = m0 + (e & 1);
+                const int col = ja + ((e >> 1) << 3);
+                const int q = (col * S) >> 7;          // owner of this column
+                const int cq = (q * 128 + S - 1) / S;  // owner's first column
+                if (m < p.M)
+                    st_dsmem_f32(&red[(rank * MP + m) * cwm + (col - cq)], static_cast<uint32_t>(q), acc[j][e]);
+            }
         }
     }
     cluster_sync_all();
     const int c0 = (rank * 128 + S - 1) / S, c1 = ((rank + 1) * 128 + S - 1) / S, cw = c1 - c0;
-    for (int o = threadIdx.x; o < cw * p.M; o += kSkThreads) {
+    for (int o = threadIdx.x; o < cw * p.M; o += kThreads) {
         const int m = o / cw, c = o - m * cw;
         const int n = nt * 128 + c0 + c;
         if (n < p.N) {
@@ -274,8 +307,11 @@ __global__ void __launch_bounds__(kSkThreads, 2) w4a16_skinny_kernel(const __gri
     }
 }
 
+// K halves per CTA: two for one token tile (one CTA per SM), one for two.
+int k_halves(int mt) { return mt == 1 ? 2 : 1; }
+
 int smem_bytes(int mt, int depth, int splits, int act_stride, int scale_rows) {
-    const int ring = depth * kSkThreads * kSlotBytes;
+    const int ring = depth * k_halves(mt) * kSkThreads * kSlotBytes;
     const int red = splits > 1 ? splits * 8 * mt * ((128 + splits - 1) / splits) * 4 : 0;
     return 8 * mt * act_stride * 2 + scale_rows * 256 + ring + red;
 }
@@ -302,7 +338,11 @@ int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan) {
     if (splits < 1) splits = 1;
     for (;;) {
         const int64_t nbmax = (KB + splits - 1) / splits;
-        const int depth = nbmax <= 4 ? 4 : 8;  // keep every block of short K ranges in flight at once
+        // Blocks in flight per thread: 8 per CTA (4 per K half with two halves),
+        // all of them for short K ranges.
+        const int64_t nbh = (nbmax + k_halves(mt) - 1) / k_halves(mt);  // blocks of one K half
+        const int dmax = 8 / k_halves(mt);
+        const int depth = nbh <= dmax / 2 ? dmax / 2 : dmax;
         const int64_t krange = nbmax * kBlockK;
         const int64_t stride = krange + 8;
         const int64_t rows = krange / G + 2;
@@ -315,6 +355,7 @@ int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan) {
             plan->scale_rows = static_cast<int>(rows < (K + G - 1) / G ? rows : (K + G - 1) / G);
             plan->smem = smem_bytes(mt, depth, plan->splits, plan->act_stride, plan->scale_rows);
             plan->mt = mt;
+            plan->threads = k_halves(mt) * kSkThreads;
             plan->grid_x = static_cast<int>(splits);
             plan->grid_y = static_cast<int>(NT);
             break;
@@ -355,10 +396,10 @@ int skinny_launch(const SkinnyPlan& plan, const void* A, const uint8_t* Wt, cons
     static bool attr_done[4][64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return W4A16_ERR_CUDA;
-    const int vi = (plan.mt - 1) * 2 + (plan.depth == 8 ? 1 : 0);
+    const int vi = (plan.mt - 1) * 2 + (plan.depth == 8 / k_halves(plan.mt) ? 1 : 0);
     // (shared-memory carve-out: the largest, so two CTAs fit per SM)
-    void (*kernels[4])(SkinnyParams) = {w4a16_skinny_kernel<1, 4>, w4a16_skinny_kernel<1, 8>,
-                                        w4a16_skinny_kernel<2, 4>, w4a16_skinny_kernel<2, 8>};
+    void (*kernels[4])(SkinnyParams) = {w4a16_skinny_kernel<1, 2, 2>, w4a16_skinny_kernel<1, 4, 2>,
+                                        w4a16_skinny_kernel<2, 4, 1>, w4a16_skinny_kernel<2, 8, 1>};
     if (!attr_done[vi][dev]) {
         if (cudaFuncSetAttribute(reinterpret_cast<const void*>(kernels[vi]),
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess ||
@@ -389,7 +430,7 @@ int skinny_launch(const SkinnyPlan& plan, const void* A, const uint8_t* Wt, cons
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(plan.grid_x), static_cast<unsigned>(plan.grid_y), 1);
-    cfg.blockDim = dim3(kSkThreads, 1, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(plan.threads), 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem);
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
