@@ -307,11 +307,14 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
     }
 }
 
-// K halves per CTA: two for one token tile (one CTA per SM), one for two.
-int k_halves(int mt) { return mt == 1 ? 2 : 1; }
+// K halves per CTA: two for one token tile over a long K range (16 or more
+// 128-deep blocks per CTA), else one. (Two halves take 512 threads and 32K
+// registers per CTA: at short K ranges the extra warps gain little, and the
+// CTA no longer fits beside a neighbouring launch's CTAs on the SM.)
+int k_halves(int mt, int64_t nbmax) { return (mt == 1 && nbmax >= 16) ? 2 : 1; }
 
-int smem_bytes(int mt, int depth, int splits, int act_stride, int scale_rows) {
-    const int ring = depth * k_halves(mt) * kSkThreads * kSlotBytes;
+int smem_bytes(int kh, int depth, int mt, int splits, int act_stride, int scale_rows) {
+    const int ring = depth * kh * kSkThreads * kSlotBytes;
     const int red = splits > 1 ? splits * 8 * mt * ((128 + splits - 1) / splits) * 4 : 0;
     return 8 * mt * act_stride * 2 + scale_rows * 256 + ring + red;
 }
@@ -340,22 +343,23 @@ int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan) {
         const int64_t nbmax = (KB + splits - 1) / splits;
         // Blocks in flight per thread: 8 per CTA (4 per K half with two halves),
         // all of them for short K ranges.
-        const int64_t nbh = (nbmax + k_halves(mt) - 1) / k_halves(mt);  // blocks of one K half
-        const int dmax = 8 / k_halves(mt);
+        const int kh = k_halves(mt, nbmax);
+        const int64_t nbh = (nbmax + kh - 1) / kh;  // blocks of one K half
+        const int dmax = 8 / kh;
         const int depth = nbh <= dmax / 2 ? dmax / 2 : dmax;
         const int64_t krange = nbmax * kBlockK;
         const int64_t stride = krange + 8;
         const int64_t rows = krange / G + 2;
-        const int64_t bytes = smem_bytes(mt, depth, static_cast<int>(splits), static_cast<int>(stride),
+        const int64_t bytes = smem_bytes(kh, depth, mt, static_cast<int>(splits), static_cast<int>(stride),
                                          static_cast<int>(rows));
         if (bytes <= 200 * 1024) {
             plan->splits = static_cast<int>(splits);
             plan->depth = depth;
             plan->act_stride = static_cast<int>(stride);
             plan->scale_rows = static_cast<int>(rows < (K + G - 1) / G ? rows : (K + G - 1) / G);
-            plan->smem = smem_bytes(mt, depth, plan->splits, plan->act_stride, plan->scale_rows);
+            plan->smem = smem_bytes(kh, depth, mt, plan->splits, plan->act_stride, plan->scale_rows);
             plan->mt = mt;
-            plan->threads = k_halves(mt) * kSkThreads;
+            plan->threads = kh * kSkThreads;
             plan->grid_x = static_cast<int>(splits);
             plan->grid_y = static_cast<int>(NT);
             break;
@@ -393,12 +397,14 @@ int skinny_device_status(bool clear) {
 
 int skinny_launch(const SkinnyPlan& plan, const void* A, const uint8_t* Wt, const void* S, void* C, int64_t M,
                   int64_t N, int64_t K, int64_t G, cudaStream_t stream) {
-    static bool attr_done[4][64] = {};
+    static bool attr_done[6][64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return W4A16_ERR_CUDA;
-    const int vi = (plan.mt - 1) * 2 + (plan.depth == 8 / k_halves(plan.mt) ? 1 : 0);
+    const int kh = plan.threads / kSkThreads;
+    const int vi = (plan.mt == 2 ? 4 : (kh == 2 ? 2 : 0)) + (plan.depth == 8 / kh ? 1 : 0);
     // (shared-memory carve-out: the largest, so two CTAs fit per SM)
-    void (*kernels[4])(SkinnyParams) = {w4a16_skinny_kernel<1, 2, 2>, w4a16_skinny_kernel<1, 4, 2>,
+    void (*kernels[6])(SkinnyParams) = {w4a16_skinny_kernel<1, 4, 1>, w4a16_skinny_kernel<1, 8, 1>,
+                                        w4a16_skinny_kernel<1, 2, 2>, w4a16_skinny_kernel<1, 4, 2>,
                                         w4a16_skinny_kernel<2, 4, 1>, w4a16_skinny_kernel<2, 8, 1>};
     if (!attr_done[vi][dev]) {
         if (cudaFuncSetAttribute(reinterpret_cast<const void*>(kernels[vi]),
