@@ -92,6 +92,19 @@ def test_shapes_and_group_sizes(o, K, N, G):
         run_dense(o, M, K, N, G, seed=K * 7 + N + G + M)
 
 
+@pytest.mark.parametrize("M,K,N,G", [
+    (5, 2176, 9480, 64),   # 17 blocks in one CTA: halves of 9 and 8; ragged last column tile
+    (8, 4160, 12288, 128),  # odd number of 64-deep tiles: the last block's second tile reads as zeros
+    (7, 8320, 4096, 32),   # 4-CTA cluster, 16-17 blocks per CTA; groups finer than a block
+    (3, 4096, 14336, 64),  # one CTA per column tile, no cluster
+])
+def test_two_k_halves_per_cta(o, M, K, N, G):
+    # one token tile over long K ranges: two sets of 8 warps split the CTA's blocks
+    rc, info = w.w4a16_gemm_launch_info(M, N, K, G)
+    assert rc == w.OK and info.threads_per_cta == 512
+    run_dense(o, M, K, N, G, seed=M + K + N + G)
+
+
 @pytest.mark.parametrize("K,N,G", [(520, 264, 48), (1032, 136, 16), (200, 392, 80)])
 def test_group_sizes_not_multiple_of_64_on_the_largest_tile(o, K, N, G):
     # 300 rows: one full 256-row tile and a ragged one; per-word scales in a stage
