@@ -78,6 +78,8 @@ class Oracle:
         lib.oracle_grouped_gemm.argtypes = [_u16p, ctypes.POINTER(_u8p), ctypes.POINTER(_u16p),
                                             _i32p, _i64, _i64, _i64, _i64, _i64, _u16p, ctypes.c_int]
         lib.oracle_grouped_gemm.restype = ctypes.c_int
+        lib.oracle_quantize.argtypes = [_u16p, _i64, _i64, _i64, _u8p, _u16p]
+        lib.oracle_quantize.restype = None
         lib.oracle_threads.restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -170,6 +172,16 @@ class Oracle:
         if rc:
             raise RuntimeError(f"oracle_grouped_gemm failed ({rc})")
         return c.view(np.float16)
+
+
+    def quantize(self, W: np.ndarray, G: int):
+        """Group-wise int4 quantisation of fp16 W [K, N]: (canonical packed codes, fp16 scales)."""
+        w = _bits(W)
+        K, N = w.shape
+        wp = np.zeros(((K + 1) // 2, N), dtype=np.uint8)
+        S = np.zeros(((K + G - 1) // G, N), dtype=np.uint16)
+        self.lib.oracle_quantize(_ptr(w, _u16p), K, N, G, _ptr(wp, _u8p), _ptr(S, _u16p))
+        return wp, S.view(np.float16)
 
 
 _default: Optional[Oracle] = None

@@ -28,7 +28,10 @@
  *       k_local = 32h + 8w + NIBBLE_K[i], NIBBLE_K = {0,2,4,6,1,3,5,7}.
  *       Codes outside [0,K) x [0,N) are 0.
  *
- * Mutants (ORACLE_MUTANT=1..12) plant one plausible mistake each; they are only
+ * Also the export step before the GEMM: group-wise symmetric int4 quantisation
+ * of fp16 weights into codes and fp16 scales (oracle_quantize, at the end).
+ *
+ * Mutants (ORACLE_MUTANT=1..15) plant one plausible mistake each; they are only
  * compiled by the oracle's own tests to show that its pins catch them.
  */
 #include <math.h>
@@ -308,4 +311,67 @@ int oracle_grouped_gemm(const uint16_t* A, const uint8_t* const* wp, const uint1
         if (rc) return rc;
     }
     return 0;
+}
+
+/* ---------------------------------------------------- weight quantisation */
+
+/*
+ * Group-wise symmetric int4 quantisation of fp16 weights W [K, N] row-major:
+ * the export step that produces the GEMM's codes and scales.
+ *
+ * The KV Cache INT8 quantization page (symmetric quantisation kernel) sets
+ * scale = max|x| / 127 and x_q = round(x / scale) in float. Here the same rule
+ * runs with the 4-bit code range (127 -> 7, the largest positive int4 code)
+ * over each group of G rows of one column (Int4 Groupwise GEMM Plugin V2 page:
+ * scales [ceil(K/G), N]), and the scale is stored in fp16 as the GEMM reads it:
+ *   amax[g, n] = max over the rows k of group g of |W[k, n]|
+ *   s[g, n]    = fp16_rne( float(amax) / 7.0f )            (IEEE float division)
+ *   q[k, n]    = clamp( round(float(W[k, n]) / float(s[g, n])), -8, 7 ),
+ *                q = 0 where s = 0
+ * with round() rounding halves away from zero, as C's round does. The codes
+ * are written in the canonical packed layout, the scales as fp16 bits.
+ * W must be finite.
+ */
+void oracle_quantize(const uint16_t* W, int64_t K, int64_t N, int64_t G, uint8_t* wp, uint16_t* S) {
+    const int64_t groups = (K + G - 1) / G;
+    memset(wp, 0, (size_t)(((K + 1) / 2) * N));
+    for (int64_t g = 0; g < groups; ++g) {
+        const int64_t k0 = g * G;
+        const int64_t k1 = k0 + G < K ? k0 + G : K;
+        for (int64_t n = 0; n < N; ++n) {
+            float amax = 0.0f;
+#if ORACLE_MUTANT == 15
+            for (int64_t k = 0; k < K; ++k) { /* the whole column instead of the group */
+#else
+            for (int64_t k = k0; k < k1; ++k) {
+#endif
+                float a = fabsf((float)oracle_half_to_double(W[k * N + n]));
+                if (a > amax) amax = a;
+            }
+#if ORACLE_MUTANT == 13
+            float s32 = amax / 8.0f; /* the int4 range taken as 8 */
+#else
+            float s32 = amax / 7.0f;
+#endif
+            uint16_t sh = oracle_double_to_half((double)s32); /* float -> double is exact */
+            S[g * N + n] = sh;
+            float s = (float)oracle_half_to_double(sh);
+            for (int64_t k = k0; k < k1; ++k) {
+                int q = 0;
+                if (s != 0.0f) {
+                    float x = (float)oracle_half_to_double(W[k * N + n]) / s;
+#if ORACLE_MUTANT == 14
+                    float r = nearbyintf(x); /* halves to even */
+#else
+                    float r = roundf(x);
+#endif
+                    q = (int)r;
+                    if (q < -8) q = -8;
+                    if (q > 7) q = 7;
+                }
+                unsigned nib = (unsigned)q & 0xF;
+                wp[(k >> 1) * N + n] |= (uint8_t)((k & 1) ? nib << 4 : nib);
+            }
+        }
+    }
 }

@@ -324,7 +324,92 @@ def pin_sample_matches_full(o) -> bool:
     return bool(np.array_equal(got.view(np.uint16), full[rows, cols].view(np.uint16)))
 
 
+def _read_quantize_example():
+    path = os.path.join(GOLDEN, "quantize_example.txt")
+    sections, cur, dims = {}, None, {}
+    with open(path) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            parts = line.split()
+            if parts[0] in ("K", "N", "G"):
+                dims[parts[0]] = int(parts[1])
+            elif parts[0] in ("W", "S", "Q"):
+                cur = parts[0]
+                sections[cur] = []
+            else:
+                sections[cur].append([float(x) for x in parts])
+    return dims, {k: np.array(v) for k, v in sections.items()}
+
+
+def pin_quantize_golden(o) -> bool:
+    """The hand-worked example: scales bit for bit, codes exactly (a tie rounds away from zero)."""
+    dims, t = _read_quantize_example()
+    W = t["W"].astype(np.float16)
+    wp, S = o.quantize(W, dims["G"])
+    q = o.unpack(wp, dims["K"])
+    return (bool(np.array_equal(S.view(np.uint16), t["S"].astype(np.float16).view(np.uint16)))
+            and bool(np.array_equal(q, t["Q"].astype(np.int8))))
+
+
+def _quantize_case(seed=21, K=200, N=24, G=64):
+    g = np.random.Generator(np.random.PCG64(seed))
+    W = (g.standard_normal((K, N)) * g.uniform(0.01, 3.0, size=(1, N))).astype(np.float16)
+    return W, K, N, G
+
+
+def pin_quantize_properties(o) -> bool:
+    """Codes in [-8, 7]; each group's largest |w| gets code +-7; |q s - w| <= s / 2 for every
+    weight (the rounding bound, with room for the float division); a partial last group."""
+    W, K, N, G = _quantize_case()
+    wp, S = o.quantize(W, G)
+    q = o.unpack(wp, K).astype(np.float64)
+    s = S.astype(np.float64)
+    w = W.astype(np.float64)
+    if q.min() < -8 or q.max() > 7:
+        return False
+    for g in range((K + G - 1) // G):
+        rows = slice(g * G, min(K, g * G + G))
+        for n in range(N):
+            col = w[rows, n]
+            if s[g, n] <= 0.0:
+                return False
+            i = int(np.argmax(np.abs(col)))
+            if abs(q[rows, n][i]) != 7 or np.sign(q[rows, n][i]) != np.sign(col[i]):
+                return False
+            if np.max(np.abs(q[rows, n] * s[g, n] - col)) > s[g, n] * (0.5 + 1e-6):
+                return False
+    return True
+
+
+def pin_quantize_scale_invariance(o) -> bool:
+    """Doubling every weight doubles every scale exactly and leaves the codes unchanged."""
+    W, K, N, G = _quantize_case(seed=22)
+    wp1, S1 = o.quantize(W, G)
+    wp2, S2 = o.quantize((W.astype(np.float32) * 2).astype(np.float16), G)
+    return (bool(np.array_equal(wp1, wp2))
+            and bool(np.array_equal(S2.astype(np.float32), 2 * S1.astype(np.float32))))
+
+
+def pin_quantize_groups_independent(o) -> bool:
+    """Changing one group's rows changes only that group's codes and scales; an all-zero group
+    gets scale 0 and codes 0."""
+    W, K, N, G = _quantize_case(seed=23)
+    wp1, S1 = o.quantize(W, G)
+    W2 = W.copy()
+    W2[G:2 * G] = 0
+    wp2, S2 = o.quantize(W2, G)
+    q1, q2 = o.unpack(wp1, K), o.unpack(wp2, K)
+    other = np.ones(K, dtype=bool)
+    other[G:2 * G] = False
+    return (bool(np.array_equal(q1[other], q2[other])) and bool(np.all(q2[G:2 * G] == 0))
+            and bool(np.all(S2[1] == 0)) and bool(np.array_equal(np.delete(S1, 1, 0), np.delete(S2, 1, 0))))
+
+
 PINS = [pin_half_widening, pin_half_rounding, pin_half_rounding_numpy, pin_pack_golden,
         pin_pack_all_bytes, pin_pack_random_odd_k, pin_tiled_positions, pin_tiled_roundtrip,
         pin_exact_small, pin_near_ties, pin_closed_form, pin_one_hot, pin_scale_duplication,
-        pin_numpy_blas, pin_grouped_segments, pin_grouped_brute, pin_sample_matches_full]
+        pin_numpy_blas, pin_grouped_segments, pin_grouped_brute, pin_sample_matches_full,
+        pin_quantize_golden, pin_quantize_properties, pin_quantize_scale_invariance,
+        pin_quantize_groups_independent]

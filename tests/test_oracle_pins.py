@@ -1,5 +1,6 @@
 """The CPU oracle against its pins (binary16 format, packing rule, exact arithmetic,
-closed forms, one-hot selection, scale duplication, numpy BLAS) and a check that
+closed forms, one-hot selection, scale duplication, numpy BLAS, the quantiser's
+worked example and properties) and a check that
 each planted mistake in the oracle breaks at least one pin."""
 import numpy as np
 import pytest
@@ -36,6 +37,9 @@ MUTANTS = {
     10: "low code not masked when packing",
     11: "tiled layout in natural nibble order",
     12: "last row of each expert segment dropped",
+    13: "quantiser scale taken as max/8",
+    14: "quantiser rounds halves to even",
+    15: "quantiser scale from the whole column",
 }
 
 
