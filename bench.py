@@ -445,10 +445,51 @@ def per_config(w4, dev):
                      "bound": "hbm" if by / (peaks["hbm_gbs"] * 1e9) >= fl / (peaks["bf16_tflops"] * 1e12)
                      else "tensor", "rotating_copies": R}
         del g
+    out["quantize"] = quantize_timing(w4, dev, peaks, l2)
     status = w4.device_status(clear=True)
     if status != w4.OK:
         raise RuntimeError(f"device status after per-config timing: {w4.status_string(status)}")
     return out
+
+
+def quantize_timing(w4, dev, peaks, l2, K=4096, N=14336, G=128):
+    """The export-time quantiser (setup, not on the GEMM path) on the MLP up projection's
+    fp16 weights: W read once, packed codes and scales written once per launch."""
+    import torch
+    gen = torch.Generator(device=dev).manual_seed(5)
+    per_w = K * N * 2
+    by = per_w + ((K + 1) // 2) * N + ((K + G - 1) // G) * N * 2
+    R = max(2, math.ceil(2 * l2 / per_w) + 1)
+    sets = []
+    for _ in range(R):
+        W = (torch.randn((K, N), generator=gen, device=dev, dtype=torch.float32) * 0.02).half()
+        sets.append((W, torch.empty(((K + 1) // 2, N), dtype=torch.uint8, device=dev),
+                     torch.empty(((K + G - 1) // G, N), dtype=torch.float16, device=dev)))
+
+    def launch(r):
+        W, wp, S = sets[r]
+        rc = w4.w4a16_quantize(W, wp, S, K, N, G)
+        if rc:
+            raise RuntimeError(w4.status_string(rc))
+    launch(0)
+    torch.cuda.synchronize()
+    n = 40
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            launch(i % R)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    e1.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / n
+    del g
+    return {"us_per_launch": round(us, 3), "GB/s": round(by / (us * 1e-6) / 1e9, 1),
+            "roofline_frac": round(by / (peaks["hbm_gbs"] * 1e9) / (us * 1e-6), 4), "bound": "hbm",
+            "rotating_copies": R, "shape": {"K": K, "N": N, "G": G}}
 
 
 # ------------------------------------------------------------------ reference arm
@@ -497,8 +538,17 @@ def run_profile(args):
     from weight_only_int4_wise_b200 import build as wbuild
     wbuild.build()
     import weight_only_int4_wise_b200 as w4
-    c = workloads.make(args.profile)
     dev = torch.device("cuda", 0)
+    if args.profile == "quantize":
+        K, N, G = 4096, 14336, 128
+        gen = torch.Generator(device=dev).manual_seed(5)
+        W = (torch.randn((K, N), generator=gen, device=dev, dtype=torch.float32) * 0.02).half()
+        for _ in range(args.launches):
+            w4.quantize(W, G)
+        torch.cuda.synchronize()
+        print(f"profiled quantize: {args.launches} launches")
+        return
+    c = workloads.make(args.profile)
     if isinstance(c, workloads.DenseCase):
         _, wt = w4.prepare_weights(torch.from_numpy(c.q).to(dev))
         A, S = torch.from_numpy(c.A).to(dev), torch.from_numpy(c.S).to(dev)
@@ -527,7 +577,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config timings")
-    ap.add_argument("--profile", choices=sorted(workloads.CONFIGS), help="only launch this workload (for ncu)")
+    ap.add_argument("--profile", choices=sorted(workloads.CONFIGS) + ["quantize"],
+                    help="only launch this workload (for ncu)")
     ap.add_argument("--launches", type=int, default=4, help="launches in --profile mode")
     args = ap.parse_args()
     if args.warmup < 3:

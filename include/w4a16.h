@@ -78,6 +78,23 @@ const char* w4a16_status_string(int status);
  * Errors: INVALID_ARG (null pointer, K <= 0, N <= 0), CUDA. */
 int w4a16_pack(const int8_t* q_dev, uint8_t* wp_dev, int64_t K, int64_t N, void* stream);
 
+/* Group-wise symmetric int4 quantisation of fp16 weights W_dev [K, N]
+ * row-major, the export step that produces the GEMM's codes and scales. Rule
+ * of the KV Cache INT8 quantization page's symmetric quantisation kernel
+ * (scale = max|x| / 127, x_q = round(x / scale)), taken with the int4 code
+ * range over each group of G rows of one column, the scale kept in fp16 as
+ * the Int4 Groupwise GEMM Plugin V2 page's scales [ceil(K/G), N]:
+ *     s[g, n] = fp16_rne(float(max |W[k, n]| over group g) / 7)
+ *     q[k, n] = clamp(round(float(W[k, n]) / float(s[g, n])), -8, 7)
+ * with IEEE float division and halves rounded away from zero; q = 0 where
+ * s = 0. Codes go to wp_dev in the canonical layout [ceil(K/2), N] (as
+ * w4a16_pack writes them), scales to S_dev [ceil(K/G), N]. W must be finite.
+ * GPU contract: N and G even, K, N < 2^31; W_dev and S_dev 4-byte aligned,
+ * wp_dev 2-byte aligned. Errors: INVALID_ARG (null pointer, K, N or G <= 0),
+ * MISALIGNED, UNSUPPORTED, CUDA. */
+int w4a16_quantize(const w4a16_half* W_dev, uint8_t* wp_dev, w4a16_half* S_dev, int64_t K, int64_t N,
+                   int64_t G, void* stream);
+
 /* Inverse of w4a16_pack: canonical wp_dev -> int8 codes q_dev [K, N], sign
  * extended. Same errors as w4a16_pack. */
 int w4a16_unpack(const uint8_t* wp_dev, int8_t* q_dev, int64_t K, int64_t N, void* stream);

@@ -97,6 +97,16 @@ def test_pack_rejects_bad_arguments_on_host(lib):
     assert w.w4a16_repack(FAKE, FAKE, 4, -4, stream=0) == w.ERR_INVALID_ARG
 
 
+def test_quantize_rejects_bad_arguments_on_host(lib):
+    q = lambda **kw: w.w4a16_quantize(kw.get("W", FAKE), kw.get("wp", FAKE), kw.get("S", FAKE), kw.get("K", 64),
+                                      kw.get("N", 64), kw.get("G", 32), stream=0)
+    assert q(W=None) == w.ERR_INVALID_ARG
+    assert q(S=None) == w.ERR_INVALID_ARG
+    assert q(K=0) == w.ERR_INVALID_ARG and q(G=-2) == w.ERR_INVALID_ARG
+    assert q(N=63) == w.ERR_UNSUPPORTED and q(G=33) == w.ERR_UNSUPPORTED
+    assert q(W=FAKE + 2) == w.ERR_MISALIGNED and q(S=FAKE + 2) == w.ERR_MISALIGNED and q(wp=FAKE + 1) == w.ERR_MISALIGNED
+
+
 def test_launch_plan_on_host(lib):
     # Nominal plans (no device here): decode runs the skinny kernel with K split across a
     # cluster (8-row token tiles for M <= 8, 16 for M <= 16); prefill tiles M on the tensor-core kernel.

@@ -190,6 +190,59 @@ def test_misaligned_pointer_is_refused():
     assert rc == w.ERR_MISALIGNED
 
 
+# --------------------------------------------------------------- quantiser
+
+def quant_case(K, N, G, seed, lo=0.01, hi=3.0, special=True):
+    g = np.random.Generator(np.random.PCG64(seed))
+    W = (g.standard_normal((K, N)) * g.uniform(lo, hi, size=(1, N))).astype(np.float16)
+    if special and K > G:  # one all-zero group in column 0 and a group of exact ties (max 3.5, w = 1.25 -> 2.5)
+        W[:G, 0] = 0
+        W[G:min(K, 2 * G), 1] = 1.25
+        W[G, 1] = 3.5
+    return W
+
+
+@pytest.mark.parametrize("K,N,G", [(200, 24, 64), (4096, 4096, 128), (7, 10, 2), (131, 66, 132), (1000, 520, 16)])
+def test_quantize_bit_exact(o, K, N, G):
+    W = quant_case(K, N, G, seed=K + N + G)
+    wp, S = w.quantize(dev(W), G)
+    torch.cuda.synchronize()
+    ref_wp, ref_S = o.quantize(W, G)
+    assert np.array_equal(S.cpu().numpy().view(np.uint16), ref_S.view(np.uint16))
+    assert np.array_equal(wp.cpu().numpy(), ref_wp)
+
+
+def test_quantize_worked_example():
+    # the hand-worked example (tests/golden/quantize_example.txt), one zero column added (N even)
+    dims, t = pins._read_quantize_example()
+    W = np.zeros((dims["K"], dims["N"] + 1), dtype=np.float16)
+    W[:, :dims["N"]] = t["W"]
+    wp, S = w.quantize(dev(W), dims["G"])
+    q = w.unpack(wp, dims["K"]).cpu().numpy()
+    torch.cuda.synchronize()
+    assert np.array_equal(q[:, :dims["N"]], t["Q"].astype(np.int8)) and np.all(q[:, -1] == 0)
+    expect = t["S"].astype(np.float16).view(np.uint16)
+    assert np.array_equal(S.cpu().numpy()[:, :dims["N"]].view(np.uint16), expect)
+
+
+def test_quantize_then_gemm(o):
+    # export path: fp16 weights -> codes and scales -> tiled layout -> GEMM. Weights of
+    # trained-model size (std 0.005-0.05 per column, scales about 0.002-0.02 as in the
+    # workloads): the GPU rounds every dequantised weight to fp16, an error that grows
+    # with |q s| and that the tolerance is sized for at these magnitudes.
+    K, N, G, M = 1024, 640, 128, 24
+    W = quant_case(K, N, G, seed=90, lo=0.005, hi=0.05, special=False)
+    A = np.random.Generator(np.random.PCG64(91)).standard_normal((M, K)).astype(np.float16)
+    wp, S = w.quantize(dev(W), G)
+    wt = w.repack(wp, K)
+    C = w.gemm(dev(A), wt, S, N, G)
+    torch.cuda.synchronize()
+    ref_wp, ref_S = o.quantize(W, G)
+    ref = o.gemm(A, ref_wp, ref_S, K, G)
+    ok, err, rel = within_tolerance(C.cpu().numpy(), ref)
+    assert ok, f"max abs err {err}, max rel err {rel}"
+
+
 # ------------------------------------------------- full-size workloads
 
 DENSE_FULL = ["decode_m1", "decode_m16", "mlp_up", "mlp_down", "mlp_up_g64"]

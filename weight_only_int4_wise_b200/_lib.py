@@ -28,7 +28,7 @@ MAX_EXPERTS = 64
 EXPORTED = [
     "w4a16_status_string", "w4a16_pack", "w4a16_unpack", "w4a16_tiled_bytes", "w4a16_repack",
     "w4a16_gemm", "w4a16_grouped_gemm", "w4a16_gemm_launch_info", "w4a16_grouped_launch_info",
-    "w4a16_device_status", "w4a16_set_static_weights",
+    "w4a16_device_status", "w4a16_set_static_weights", "w4a16_quantize",
 ]
 
 
@@ -66,6 +66,8 @@ def load() -> ctypes.CDLL:
             f = getattr(lib, name)
             f.argtypes = [_vp, _vp, _i64, _i64, _vp]
             f.restype = ctypes.c_int
+        lib.w4a16_quantize.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp]
+        lib.w4a16_quantize.restype = ctypes.c_int
         lib.w4a16_tiled_bytes.argtypes = [_i64, _i64]
         lib.w4a16_tiled_bytes.restype = _i64
         lib.w4a16_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]
@@ -126,6 +128,10 @@ def _check(status: int, where: str) -> None:
 
 def w4a16_pack(q, wp, K: int, N: int, stream=None) -> int:
     return load().w4a16_pack(_addr(q), _addr(wp), K, N, _stream(stream))
+
+
+def w4a16_quantize(W, wp, S, K: int, N: int, G: int, stream=None) -> int:
+    return load().w4a16_quantize(_addr(W), _addr(wp), _addr(S), K, N, G, _stream(stream))
 
 
 def w4a16_unpack(wp, q, K: int, N: int, stream=None) -> int:
@@ -189,6 +195,20 @@ def pack(q, stream=None):
     wp = torch.empty(((K + 1) // 2, N), dtype=torch.uint8, device=q.device)
     _check(w4a16_pack(q.contiguous(), wp, K, N, stream), "w4a16_pack")
     return wp
+
+
+def quantize(W, G: int, stream=None):
+    """fp16 weights [K, N] (device) -> (canonical packed codes [ceil(K/2), N] uint8,
+    fp16 scales [ceil(K/G), N]): group-wise symmetric int4 quantisation."""
+    import torch
+    _require_cuda(W)
+    if W.dtype != torch.float16:
+        raise TypeError("W must be float16")
+    K, N = W.shape
+    wp = torch.empty(((K + 1) // 2, N), dtype=torch.uint8, device=W.device)
+    S = torch.empty(((K + G - 1) // G, N), dtype=torch.float16, device=W.device)
+    _check(w4a16_quantize(W.contiguous(), wp, S, K, N, G, stream), "w4a16_quantize")
+    return wp, S
 
 
 def unpack(wp, K: int, stream=None):

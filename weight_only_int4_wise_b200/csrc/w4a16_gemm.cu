@@ -785,6 +785,20 @@ void fill_info(const Plan& plan, w4a16_launch_info* info) {
 
 }  // namespace
 
+int make_half_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                     uint32_t box_inner, uint32_t box_outer) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return W4A16_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
 int check_device() {
     // per device: 0 unknown, 1 supported, 2 not (cached: this runs on every call)
     static std::atomic<int> state[64];
@@ -988,6 +1002,7 @@ extern "C" int w4a16_device_status(int clear) {
         if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return W4A16_ERR_CUDA;
     }
     const int vs = skinny_device_status(clear != 0);
-    if (vs < 0) return W4A16_ERR_CUDA;
-    return v != 0 ? v : vs;
+    const int vq = quant_device_status(clear != 0);
+    if (vs < 0 || vq < 0) return W4A16_ERR_CUDA;
+    return v != 0 ? v : (vs != 0 ? vs : vq);
 }

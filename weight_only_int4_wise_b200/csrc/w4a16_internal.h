@@ -1,6 +1,7 @@
 // Host-side helpers shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -18,6 +19,15 @@ int sm_count();
 
 // Whether the caller declared weights and scales static (w4a16_set_static_weights).
 bool static_weights_enabled();
+
+// A tiled tensor map over fp16 elements [outer, inner] (row stride in bytes),
+// box [box_outer, box_inner], no swizzle, zero fill outside the tensor.
+// W4A16_OK, or W4A16_ERR_CUDA if the driver's encoder is missing or refuses.
+int make_half_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                     uint32_t box_inner, uint32_t box_outer);
+
+// The quantiser kernel's latched device status (0 = none, -1 if it could not be read).
+int quant_device_status(bool clear);
 
 // Decode-sized products (M <= kSkinnyMaxM) run on the skinny kernel.
 constexpr int kSkinnyMaxM = 16;
