@@ -112,6 +112,11 @@ def test_launch_plan_on_host(lib):
     # cluster (8-row token tiles for M <= 8, 16 for M <= 16); prefill tiles M on the tensor-core kernel.
     rc, info = w.w4a16_gemm_launch_info(1, 4096, 4096, 128)
     assert rc == w.OK and info.token_tile == 8 and info.k_splits > 1 and info.grid_y == 32
+    assert info.threads_per_cta == 256  # decode keeps one set of 8 warps per CTA
+    rc, info = w.w4a16_gemm_launch_info(8, 14336, 4096, 128)
+    assert rc == w.OK and info.token_tile == 8 and info.threads_per_cta == 512  # MLP up: two K halves
+    rc, info = w.w4a16_gemm_launch_info(8, 4096, 14336, 128)
+    assert rc == w.OK and info.k_splits == 4 and info.threads_per_cta == 512  # MLP down: 28 blocks per CTA
     rc, info = w.w4a16_gemm_launch_info(16, 4096, 4096, 128)
     assert rc == w.OK and info.token_tile == 16 and info.threads_per_cta == 256
     rc, info = w.w4a16_gemm_launch_info(17, 4096, 4096, 128)
