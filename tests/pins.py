@@ -407,9 +407,21 @@ def pin_quantize_groups_independent(o) -> bool:
             and bool(np.all(S2[1] == 0)) and bool(np.array_equal(np.delete(S1, 1, 0), np.delete(S2, 1, 0))))
 
 
+def pin_quantize_edges(o) -> bool:
+    """Odd K: the last packed row's high nibbles are 0. A group whose largest |w| is below
+    3.5 * 2^-24 (half the smallest fp16 step, times 7) rounds its scale to 0 and its codes to 0."""
+    W = np.array([[0.5, -0.25], [0.125, 1.0], [-1.0, 0.0], [2.0, -3.0], [1.5, 0.75]], dtype=np.float16)
+    wp, S = o.quantize(W, 2)
+    if wp.shape != (3, 2) or np.any(wp[2] >> 4):
+        return False
+    tiny = np.array([[2.0 ** -24, -2.0 ** -24], [0.0, 2.0 ** -23]], dtype=np.float16)  # max 2^-23 < 3.5 * 2^-24
+    wp_t, S_t = o.quantize(tiny, 2)
+    return bool(np.all(S_t.view(np.uint16) == 0)) and bool(np.all(wp_t == 0))
+
+
 PINS = [pin_half_widening, pin_half_rounding, pin_half_rounding_numpy, pin_pack_golden,
         pin_pack_all_bytes, pin_pack_random_odd_k, pin_tiled_positions, pin_tiled_roundtrip,
         pin_exact_small, pin_near_ties, pin_closed_form, pin_one_hot, pin_scale_duplication,
         pin_numpy_blas, pin_grouped_segments, pin_grouped_brute, pin_sample_matches_full,
         pin_quantize_golden, pin_quantize_properties, pin_quantize_scale_invariance,
-        pin_quantize_groups_independent]
+        pin_quantize_groups_independent, pin_quantize_edges]
