@@ -64,8 +64,10 @@ __device__ __forceinline__ __half2 group_scales(float a0, float a1) {
     return __halves2half2(__float2half_rn(__fdiv_rn(a0, 7.0f)), __float2half_rn(__fdiv_rn(a1, 7.0f)));
 }
 
-// One group (rows k0..k1) of column pair c from `rows` (a row stride of `stride`
-// half2): the scales, then the packed bytes of every row pair.
+// Rows 0..nrows-1 of one column pair, read through row(r), whose maxima are
+// (a0, a1): the pair's fp16 scales (stored at s_out), then one packed byte per
+// column and row pair, written from wp_row0 on with a stride of N2 16-bit words
+// per packed row.
 template <typename RowFn>
 __device__ __forceinline__ void quantize_pair(RowFn row, int64_t nrows, uint16_t* __restrict__ wp_row0,
                                               int64_t N2, __half2* __restrict__ s_out, float a0, float a1) {
