@@ -294,6 +294,16 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
     return r;
 }
 
+// Split form of the cluster barrier: arrive (no ordering of this thread's
+// memory operations), then later wait for every thread of the cluster to arrive.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

@@ -151,6 +151,9 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
     }
     cp_async_wait<kDepth - 1>();  // the scale rows (and this thread's first block) have landed
     __syncthreads();              // staged activations and scale rows are visible to all threads
+    // Distributed shared memory may be written only once every CTA of the cluster
+    // has started: arrive here, and wait for the others before the first remote store.
+    if (p.splits > 1) cluster_arrive_relaxed();
 
     float acc[MT][4], acc2[MT][4];  // (acc2: the odd-step chain when groups are finer than a block)
 #pragma unroll
@@ -279,6 +282,7 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
     // [ceil(q*128/S), ceil((q+1)*128/S))), one cluster barrier publishes them,
     // and each owner sums its S slices in rank order.
     const int rank = static_cast<int>(cluster_ctarank());
+    cluster_wait();
     if (kh == 0) {
 #pragma unroll
         for (int j = 0; j < MT; ++j) {
