@@ -162,6 +162,20 @@ int w4a16_gemm_launch_info(int64_t M, int64_t N, int64_t K, int64_t G, w4a16_lau
 int w4a16_grouped_launch_info(int64_t E, int64_t total_rows, int64_t N, int64_t K, int64_t G,
                               w4a16_launch_info* info);
 
+/* Test aid for the failure path of the bounded device waits (no counterpart
+ * on the plugin pages). For every later launch of the tensor-core GEMM kernel
+ * (w4a16_gemm with M > 16, and w4a16_grouped_gemm) until it is called again:
+ * every bounded wait in the kernel runs out after wait_limit_cycles SM clock
+ * cycles (<= 0 restores the default of about 2 s), and, if stall_stage >= 0,
+ * the dequantising warps withhold the ready signal of that 64-deep K stage
+ * (counted from the start of each CTA's K range), so the MMA thread's wait for
+ * it runs out. The kernel then latches W4A16_ERR_TIMEOUT, lets every copy and
+ * MMA in flight complete, frees its tensor memory and writes no output tile
+ * that the stalled stage (or, with K split over a cluster, any CTA of the
+ * cluster) contributes to; nothing faults or hangs. Process-wide; always
+ * returns W4A16_OK. */
+int w4a16_set_fault_injection(int64_t stall_stage, int64_t wait_limit_cycles);
+
 /* Reads (and, if clear != 0, resets) the current device's status word. This
  * synchronizes the current device. Returns W4A16_OK, W4A16_ERR_TIMEOUT,
  * W4A16_ERR_BAD_OFFSETS, or W4A16_ERR_CUDA if the read itself failed. */

@@ -92,16 +92,47 @@ def test_shapes_and_group_sizes(o, K, N, G):
 
 
 @pytest.mark.parametrize("M,K,N,G", [
-    (5, 2176, 9480, 64),   # 17 blocks in one CTA: halves of 9 and 8; ragged last column tile
-    (8, 4160, 12288, 128),  # odd number of 64-deep tiles: the last block's second tile reads as zeros
+    (5, 2176, 9480, 48),   # 17 blocks in one CTA: halves of 9 and 8; ragged last column tile
+    (8, 4160, 12288, 16),  # odd number of 64-deep tiles: the last block's second tile reads as zeros
     (7, 8320, 4096, 32),   # 4-CTA cluster, 16-17 blocks per CTA; groups finer than a block
-    (3, 4096, 14336, 64),  # one CTA per column tile, no cluster
+    (3, 4096, 14336, 80),  # one CTA per column tile, no cluster
 ])
 def test_two_k_halves_per_cta(o, M, K, N, G):
-    # one token tile over long K ranges: two sets of 8 warps split the CTA's blocks
+    # G not a multiple of 64 runs the warp-MMA skinny kernel; one token tile over long
+    # K ranges: two sets of 8 warps split the CTA's blocks
     rc, info = w.w4a16_gemm_launch_info(M, N, K, G)
     assert rc == w.OK and info.threads_per_cta == 512
     run_dense(o, M, K, N, G, seed=M + K + N + G)
+
+
+@pytest.mark.parametrize("M,K,N,G", [
+    (1, 4096, 4096, 128),   # 4-CTA clusters, 16 stages per CTA (more than the 14-stage ring)
+    (16, 4096, 4096, 64),   # one scale group per stage
+    (3, 1000, 392, 128),    # K % 64 != 0 (zero-padded last stage), ragged last column tile
+    (8, 8192, 1024, 256),   # 8-CTA clusters; groups of four stages
+    (5, 2048, 136, 2048),   # one group per CTA range; 8 CTAs per cluster
+    (16, 960, 8, 64),       # a single 8-column tile, 15 stages split 8 ways
+    (2, 192, 264, 4096),    # G > K: one group
+    (12, 14336, 256, 128),  # long K ranges: every ring wraps several times
+    (7, 4160, 12288, 128),  # 96 column tiles, one CTA per tile: 65 stages per CTA
+])
+def test_skinny_kernel_more_shapes(o, M, K, N, G):
+    # decode-sized M with G a multiple of 64: clusters of 1 to 8 CTAs, ragged K and N,
+    # one group per CTA range, long K ranges that wrap every ring
+    rc, info = w.w4a16_gemm_launch_info(M, N, K, G)
+    assert rc == w.OK and info.token_tile in (8, 16)  # the skinny kernel
+    run_dense(o, M, K, N, G, seed=M * 31 + K + N + G)
+
+
+def test_skinny_long_k_with_large_activations(o):
+    # |A| ~ 8 over K = 14336: partial sums of tens of units stay within tolerance
+    run_dense(o, 16, 14336, 256, 128, seed=78, a_scale=8.0)
+
+
+@pytest.mark.parametrize("M", [2, 9, 16])
+def test_skinny_kernel_two_token_tiles(o, M):
+    # G = 48: the warp-MMA skinny kernel, one and two 8-row token tiles, ragged tiles
+    run_dense(o, M, 1040, 392, 48, seed=900 + M)
 
 
 @pytest.mark.parametrize("K,N,G", [(520, 264, 48), (1032, 136, 16), (200, 392, 80)])

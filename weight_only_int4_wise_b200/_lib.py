@@ -28,7 +28,7 @@ MAX_EXPERTS = 64
 EXPORTED = [
     "w4a16_status_string", "w4a16_pack", "w4a16_unpack", "w4a16_tiled_bytes", "w4a16_repack",
     "w4a16_gemm", "w4a16_grouped_gemm", "w4a16_gemm_launch_info", "w4a16_grouped_launch_info",
-    "w4a16_device_status", "w4a16_set_static_weights", "w4a16_quantize",
+    "w4a16_device_status", "w4a16_set_static_weights", "w4a16_quantize", "w4a16_set_fault_injection",
 ]
 
 
@@ -83,6 +83,8 @@ def load() -> ctypes.CDLL:
         lib.w4a16_device_status.restype = ctypes.c_int
         lib.w4a16_set_static_weights.argtypes = [ctypes.c_int]
         lib.w4a16_set_static_weights.restype = ctypes.c_int
+        lib.w4a16_set_fault_injection.argtypes = [_i64, _i64]
+        lib.w4a16_set_fault_injection.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -177,6 +179,11 @@ def w4a16_device_status(clear: bool = True) -> int:
 def w4a16_set_static_weights(enable: bool) -> int:
     """Declare weights and scales static (see include/w4a16.h); returns the previous setting."""
     return int(load().w4a16_set_static_weights(1 if enable else 0))
+
+
+def w4a16_set_fault_injection(stall_stage: int, wait_limit_cycles: int) -> int:
+    """Test aid: stall one K stage and bound every device wait (see include/w4a16.h)."""
+    return int(load().w4a16_set_fault_injection(int(stall_stage), int(wait_limit_cycles)))
 
 
 # ------------------------------------------------------------- torch helpers

@@ -81,6 +81,8 @@ struct Params {
     int32_t grouped;
     int32_t prefetch;   // weights/scales may be read before the previous kernel finishes
     int32_t vec_out;    // C rows start on 16-byte boundaries (16-byte output stores)
+    long long wait_limit;   // bound of every device wait, in SM clock cycles
+    int32_t stall_stage;    // test aid: the dequantising warps withhold this stage's ready signal (< 0: never)
 };
 
 // One ring of LS stages. Stage s owns, in shared memory, an activation tile
@@ -113,7 +115,7 @@ __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0,
 // the wait ran out (which starts the abort). The bound is counted in SM clock
 // cycles (clock64 is a cheap, SM-local register; the global timer is far slower
 // to read and would add its latency to every pipeline hand-off).
-__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag, long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     long long start = 0;
     for (uint32_t it = 1;; ++it) {
@@ -123,7 +125,7 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volat
             const long long now = clock64();
             if (start == 0) {
                 start = now;
-            } else if (now - start > kTimeoutCycles) {
+            } else if (now - start > limit) {
                 *abort_flag = 1;
                 latch_status(W4A16_ERR_TIMEOUT);
                 return false;
@@ -135,6 +137,7 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volat
 // Bounded wait that ignores the abort flag: used where in-flight asynchronous
 // work must finish before its resources are released.
 __device__ __forceinline__ bool drain_phase(uint64_t* bar, uint32_t parity) {
+    const long long limit = kTimeoutCycles;  // drains keep the long bound whatever the wait bound is
     long long start = 0;
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -142,7 +145,7 @@ __device__ __forceinline__ bool drain_phase(uint64_t* bar, uint32_t parity) {
             const long long now = clock64();
             if (start == 0) {
                 start = now;
-            } else if (now - start > kTimeoutCycles) {
+            } else if (now - start > limit) {
                 latch_status(W4A16_ERR_TIMEOUT);
                 return false;
             }
@@ -154,19 +157,21 @@ __device__ __forceinline__ bool drain_phase(uint64_t* bar, uint32_t parity) {
 // the whole warp), then every lane observes the completed phase itself, which
 // gives each lane acquire ordering on the data the phase guards. The phase
 // cannot move on before this warp arrives elsewhere, so that check is immediate.
-__device__ __forceinline__ bool warp_wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool warp_wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                long long limit) {
     int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = wait_phase(bar, parity, abort_flag) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_phase(bar, parity, abort_flag, limit) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (ok) mbar_try_wait(bar, parity);
     return ok != 0;
 }
 
-__device__ __forceinline__ void warp_drain_phase(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool warp_drain_phase(uint64_t* bar, uint32_t parity) {
     int ok = 0;
     if ((threadIdx.x & 31) == 0) ok = drain_phase(bar, parity) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (ok) mbar_try_wait(bar, parity);
+    return ok != 0;
 }
 
 // OG: G is a multiple of 64, so a stage lies inside one scale group.
@@ -343,7 +348,8 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             int issued = first;
             for (; issued < nst; ++issued) {
                 const int i = issued;
-                if (i >= LS && !wait_phase(&done[i % LS], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
+                if (i >= LS &&
+                    !wait_phase(&done[i % LS], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag, p.wait_limit))
                     break;
                 issue_act(i);
                 if (i + kPrefetchStages < nst)
@@ -370,7 +376,7 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
                 for (int qq = 0; qq < LS / 2; ++qq) {
                     const int i = base + 2 * qq;
                     if (i >= nst) break;
-                    if (!wait_phase(&afull[qq], par, abort_flag)) {
+                    if (!wait_phase(&afull[qq], par, abort_flag, p.wait_limit)) {
                         stop = true;
                         break;
                     }
@@ -413,7 +419,8 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             }
             load_next(r, sv);
             // (Columns past N hold code 0 in the tiled layout and get scale 0: v is 0.)
-            if (i >= LS && !warp_wait_phase(&done[s], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag))
+            if (i >= LS &&
+                !warp_wait_phase(&done[s], static_cast<uint32_t>((i / LS) - 1) & 1u, abort_flag, p.wait_limit))
                 return false;
             tc_fence_after_sync();
             tmem_st_32x32b_x16(tmem_ring + tlane + s * kSlotCols, v[0]);
@@ -423,10 +430,12 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             // The group's first warp also sees the stage's activation tile land,
             // so that the MMA thread waits on one barrier per stage pair. The
             // last stage of an odd count arrives for its missing partner too.
-            if ((dw & 3) == 0 && !warp_wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag))
+            if ((dw & 3) == 0 &&
+                !warp_wait_phase(&full[s], static_cast<uint32_t>(i / LS) & 1u, abort_flag, p.wait_limit))
                 return false;
             __syncwarp();
-            if (lane == 0) mbar_arrive_cnt(&afull[(i >> 1) % (LS / 2)], ((i & 1) == 0 && i + 1 == nst) ? 2u : 1u);
+            if (lane == 0 && i != p.stall_stage)
+                mbar_arrive_cnt(&afull[(i >> 1) % (LS / 2)], ((i & 1) == 0 && i + 1 == nst) ? 2u : 1u);
             return true;
         };
         // kAhead = 2 register slots, used alternately: a stage's codes stay in
@@ -441,11 +450,11 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         // -------------------------------------------------- epilogue
         // The accumulator is complete (or the CTA is aborting) once accfull fires;
         // either way no MMA may still run when TMEM is released.
-        warp_drain_phase(accfull, 0);
+        const bool drained = warp_drain_phase(accfull, 0);
         tc_fence_after_sync();
         grid_dependency_wait();  // the output may still be read by the previous kernel
         const int aborted = __shfl_sync(0xffffffffu, *abort_flag, 0);
-        const bool have_acc = !aborted && nst > 0;
+        const bool have_acc = drained && !aborted && nst > 0;
         if (dw == 0 && lane == 0) tile_info[4] = have_acc ? 1 : 0;
         if (p.splits == 1) {
             // Stage the fp16 tile, row-major [token][128 columns], in the idle
@@ -519,7 +528,11 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         const int cw = kTileN / S;
         const int rank = static_cast<int>(cluster_ctarank());
         const float* red = reinterpret_cast<const float*>(smem + L::kAct);
-        const bool aborted = *abort_flag != 0;
+        // A CTA that stopped early left its partial tile incomplete: if any CTA of
+        // the cluster did, none writes the tile.
+        bool aborted = false;
+        for (int src = 0; src < S; ++src)
+            aborted |= __float_as_int(ld_dsmem_f32(const_cast<int*>(abort_flag), static_cast<uint32_t>(src))) != 0;
         for (int o = threadIdx.x; o < cw * rows; o += static_cast<int>(blockDim.x)) {
             const int col = rank * cw + (o % cw);
             const int tok = o / cw;
@@ -757,19 +770,6 @@ int plan_grouped(int64_t E, int64_t total_rows, int64_t N, int64_t K, Plan* plan
     return W4A16_OK;
 }
 
-int make_act_map(CUtensorMap* map, const void* A, int64_t rows, int64_t K, int bn) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return W4A16_ERR_CUDA;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(bn)};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(A), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? W4A16_OK : W4A16_ERR_CUDA;
-}
-
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 void fill_info(const Plan& plan, w4a16_launch_info* info) {
@@ -784,6 +784,49 @@ void fill_info(const Plan& plan, w4a16_launch_info* info) {
 }
 
 }  // namespace
+
+int activation_map(CUtensorMap* map, const void* A, int64_t rows, int64_t K, int box_rows) {
+    // A small per-thread cache: the encoder costs more than the rest of a
+    // decode-sized call on the host, and the same activation buffers recur.
+    struct Entry {
+        const void* A;
+        int64_t rows, K;
+        int box, dev;
+        CUtensorMap map;
+    };
+    constexpr int kEntries = 16;
+    thread_local Entry cache[kEntries];
+    thread_local int used = 0, next = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W4A16_ERR_CUDA;
+    for (int i = 0; i < used; ++i) {
+        const Entry& e = cache[i];
+        if (e.A == A && e.rows == rows && e.K == K && e.box == box_rows && e.dev == dev) {
+            *map = e.map;
+            return W4A16_OK;
+        }
+    }
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return W4A16_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(A), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return W4A16_ERR_CUDA;
+    Entry& e = cache[next];
+    e.A = A;
+    e.rows = rows;
+    e.K = K;
+    e.box = box_rows;
+    e.dev = dev;
+    e.map = *map;
+    next = (next + 1) % kEntries;
+    if (used < kEntries) ++used;
+    return W4A16_OK;
+}
 
 int make_half_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                      uint32_t box_inner, uint32_t box_outer) {
@@ -823,6 +866,8 @@ int check_device() {
 
 namespace {
 std::atomic<int> g_static_weights{0};
+std::atomic<long long> g_wait_limit{kTimeoutCycles};  // test aid: w4a16_set_fault_injection
+std::atomic<int> g_stall_stage{-1};
 }
 
 bool static_weights_enabled() { return g_static_weights.load(std::memory_order_relaxed) != 0; }
@@ -935,9 +980,11 @@ extern "C" int w4a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt_dev, const 
     p.grouped = 0;
     p.prefetch = static_weights_enabled() ? 1 : 0;
     p.vec_out = (N % 8) == 0 && aligned16(C_dev);
+    p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
+    p.stall_stage = g_stall_stage.load(std::memory_order_relaxed);
 
     CUtensorMap map;
-    rc = make_act_map(&map, A_dev, M, K, plan.bn);
+    rc = activation_map(&map, A_dev, M, K, plan.bn);
     if (rc) return rc;
     const Variant& v = variant_for(plan.bn);
     return v.launch[(G % kTileK) ? 1 : 0](map, p, plan.grid, plan.splits, v.smem, static_cast<cudaStream_t>(stream));
@@ -984,9 +1031,11 @@ extern "C" int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const*
     p.grouped = 1;
     p.vec_out = (N % 8) == 0 && aligned16(C_dev);
     p.prefetch = 0;  // expert weights are read only after the offsets, which follow the wait
+    p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
+    p.stall_stage = g_stall_stage.load(std::memory_order_relaxed);
 
     CUtensorMap map;
-    rc = make_act_map(&map, A_dev, total_rows, K, plan.bn);
+    rc = activation_map(&map, A_dev, total_rows, K, plan.bn);
     if (rc) return rc;
     const Variant& v = variant_for(plan.bn);
     return v.launch[(G % kTileK) ? 1 : 0](map, p, plan.grid, 1, v.smem, static_cast<cudaStream_t>(stream));
@@ -1005,4 +1054,10 @@ extern "C" int w4a16_device_status(int clear) {
     const int vq = quant_device_status(clear != 0);
     if (vs < 0 || vq < 0) return W4A16_ERR_CUDA;
     return v != 0 ? v : (vs != 0 ? vs : vq);
+}
+
+extern "C" int w4a16_set_fault_injection(int64_t stall_stage, int64_t wait_limit_cycles) {
+    g_stall_stage.store(stall_stage < 0 || stall_stage > (1 << 30) ? -1 : static_cast<int>(stall_stage));
+    g_wait_limit.store(wait_limit_cycles > 0 ? static_cast<long long>(wait_limit_cycles) : kTimeoutCycles);
+    return W4A16_OK;
 }

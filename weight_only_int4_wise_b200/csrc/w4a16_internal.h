@@ -26,6 +26,13 @@ bool static_weights_enabled();
 int make_half_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                      uint32_t box_inner, uint32_t box_outer);
 
+// A tiled tensor map over activations A [rows, K] fp16 with a {64, box_rows}
+// box, the 128-byte swizzle and zero fill past the tensor, as the tensor-core
+// kernels stage them. Encoded maps are kept in a small per-thread cache keyed
+// by (device, address, rows, K, box_rows), so repeated calls on the same
+// buffers skip the encoder.
+int activation_map(CUtensorMap* map, const void* A, int64_t rows, int64_t K, int box_rows);
+
 // The quantiser kernel's latched device status (0 = none, -1 if it could not be read).
 int quant_device_status(bool clear);
 
