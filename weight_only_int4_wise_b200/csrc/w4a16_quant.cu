@@ -114,9 +114,11 @@ __global__ void __launch_bounds__(kQuantThreads * kSlices) quantize_tma_kernel(c
         if (threadIdx.x == 0) {
             mbar_arrive_expect_tx(bar, static_cast<uint32_t>(G * kTileCols * 2));
             tma_load_2d(const_cast<__half2*>(tile), &tmW, static_cast<int32_t>(blockIdx.x) * kTileCols, static_cast<int32_t>(k0), bar);
-            // Bounded wait for the copy. Past the bound the status is latched, the
-            // copy gets a second bound to land (shared memory must not be released
-            // under it), and the whole CTA stops.
+            // Bounded wait for the copy. Past the first bound the status is latched
+            // and the copy gets a second bound to land. If it has still not landed
+            // then, the whole CTA stops with the copy possibly still in flight into
+            // its shared memory: the latched status is then the only signal, and
+            // the CTA's output tile is not written.
             long long start = 0;
             int bounds = 0;
             for (uint32_t it = 0; !mbar_try_wait(bar, phase); ++it) {
