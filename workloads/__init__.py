@@ -106,6 +106,38 @@ def grouped(E: int, top_k: int, tokens: int, K: int, N: int, G: int, seed: int,
                        order.astype(np.int64), np.ascontiguousarray(A), offsets, q, S)
 
 
+@dataclasses.dataclass
+class MoeCase:
+    name: str
+    tokens: int
+    E: int
+    top_k: int
+    H: int
+    I: int
+    G: int
+    seed: int
+    X: np.ndarray         # [tokens, H] float16 hidden states
+    logits: np.ndarray    # [tokens, E] float16 router logits
+    q_up: np.ndarray      # [E, H, I] int8 codes of the up projections
+    S_up: np.ndarray      # [E, ceil(H/G), I] float16
+    q_down: np.ndarray    # [E, I, H] int8 codes of the down projections
+    S_down: np.ndarray    # [E, ceil(I/G), H] float16
+
+
+def moe(tokens: int, E: int, top_k: int, H: int, I: int, G: int, seed: int, name: str = "moe") -> MoeCase:
+    """A mixture-of-experts layer case (Int4MoePlugin page, constructor: numExperts,
+    topK, hiddenSize, moeInterSize, quantizationGroupSize): hidden states and router
+    logits ~ N(0, 1) rounded to fp16; per-expert codes and scales as in `dense`."""
+    g = _rng(seed)
+    X = g.standard_normal((tokens, H), dtype=np.float32).astype(np.float16)
+    logits = g.standard_normal((tokens, E), dtype=np.float32).astype(np.float16)
+    q_up = g.integers(-8, 8, size=(E, H, I), dtype=np.int8)
+    S_up = g.uniform(S_LOW, S_HIGH, size=(E, n_groups(H, G), I)).astype(np.float32).astype(np.float16)
+    q_down = g.integers(-8, 8, size=(E, I, H), dtype=np.int8)
+    S_down = g.uniform(S_LOW, S_HIGH, size=(E, n_groups(I, G), H)).astype(np.float32).astype(np.float16)
+    return MoeCase(name, tokens, E, top_k, H, I, G, seed, X, logits, q_up, S_up, q_down, S_down)
+
+
 # The five workload families and their sizes, with a fixed seed per config.
 CONFIGS: Dict[str, dict] = {
     "tiny":        dict(kind="dense", M=4, K=512, N=512, G=128, seed=0),
@@ -116,6 +148,9 @@ CONFIGS: Dict[str, dict] = {
     "mlp_up_g64":  dict(kind="dense", M=8, K=4096, N=14336, G=64, seed=22),
     "prefill":     dict(kind="dense", M=2048, K=4096, N=4096, G=128, seed=3),
     "grouped":     dict(kind="grouped", E=8, top_k=2, tokens=512, K=4096, N=14336, G=128, seed=4),
+    # the whole mixture-of-experts layer around the grouped product (up 4096 -> 14336,
+    # down 14336 -> 4096), routed by its own logits
+    "moe_layer":   dict(kind="moe", E=8, top_k=2, tokens=512, H=4096, I=14336, G=128, seed=6),
 }
 
 
@@ -124,4 +159,6 @@ def make(name: str):
     kind = cfg.pop("kind")
     if kind == "dense":
         return dense(name=name, **cfg)
+    if kind == "moe":
+        return moe(name=name, **cfg)
     return grouped(name=name, **cfg)
