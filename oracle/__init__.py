@@ -80,6 +80,12 @@ class Oracle:
         lib.oracle_grouped_gemm.restype = ctypes.c_int
         lib.oracle_quantize.argtypes = [_u16p, _i64, _i64, _i64, _u8p, _u16p]
         lib.oracle_quantize.restype = None
+        lib.oracle_tiled_bytes_w8.argtypes = [_i64, _i64]
+        lib.oracle_tiled_bytes_w8.restype = _i64
+        lib.oracle_tile_w8.argtypes = [_i8p, _i64, _i64, _u8p]
+        lib.oracle_tile_w8.restype = None
+        lib.oracle_gemm_w8.argtypes = [_u16p, _i8p, _u16p, _i64, _i64, _i64, _i64, _u16p, ctypes.c_int]
+        lib.oracle_gemm_w8.restype = ctypes.c_int
         lib.oracle_threads.restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -173,6 +179,33 @@ class Oracle:
             raise RuntimeError(f"oracle_grouped_gemm failed ({rc})")
         return c.view(np.float16)
 
+
+    # -- the 8-bit code variant (W8A16) ----------------------------------
+    def tiled_bytes_w8(self, K: int, N: int) -> int:
+        return int(self.lib.oracle_tiled_bytes_w8(K, N))
+
+    def tile_w8(self, q8: np.ndarray) -> np.ndarray:
+        q8 = np.ascontiguousarray(q8, dtype=np.int8)
+        K, N = q8.shape
+        wt = np.empty(self.tiled_bytes_w8(K, N), dtype=np.uint8)
+        self.lib.oracle_tile_w8(_ptr(q8, _i8p), K, N, _ptr(wt, _u8p))
+        return wt
+
+    def gemm_w8(self, A: np.ndarray, q8: np.ndarray, S: np.ndarray, K: int, G: int,
+                threads: int = 0) -> np.ndarray:
+        """C = fp16(A @ (q8 * s)) for signed 8-bit codes q8 [K, N]."""
+        a = _bits(A)
+        s = _bits(S)
+        q8 = np.ascontiguousarray(q8, dtype=np.int8)
+        M = a.shape[0]
+        N = q8.shape[1]
+        assert a.shape == (M, K) and q8.shape == (K, N) and s.shape == (-(-K // G), N)
+        c = np.zeros((M, N), dtype=np.uint16)
+        rc = self.lib.oracle_gemm_w8(_ptr(a, _u16p), _ptr(q8, _i8p), _ptr(s, _u16p), M, N, K, G,
+                                     _ptr(c, _u16p), int(threads))
+        if rc:
+            raise RuntimeError(f"oracle_gemm_w8 failed ({rc})")
+        return c.view(np.float16)
 
     def quantize(self, W: np.ndarray, G: int):
         """Group-wise int4 quantisation of fp16 W [K, N]: (canonical packed codes, fp16 scales)."""

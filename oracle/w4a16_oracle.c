@@ -375,3 +375,92 @@ void oracle_quantize(const uint16_t* W, int64_t K, int64_t N, int64_t G, uint8_t
         }
     }
 }
+
+/* ------------------------------------------------ W8A16 (8-bit codes) */
+
+/*
+ * The INT8 weight-only variant (the FP8-vs-INT8 TensorRT-LLM comparison page
+ * lists INT8 weight-only with an FP16 KV cache among the INT8 configurations):
+ * the same group-wise product with signed 8-bit codes in [-128, 127], one per
+ * byte, q8 [K, N] row-major (two's complement):
+ *     C[m, n] = fp16_rne( sum_{k < K} A[m, k] * q8[k, n] * s[floor(k / G), n] )
+ * summed in double in increasing k and rounded once, as oracle_gemm.
+ *
+ * Tiled layout of 8-bit codes (the library's W8 weight operand):
+ * ceil(N/128) x ceil(K/64) tiles of 8192 bytes, tile (nt, kt) at byte
+ * ((nt * KT) + kt) * 8192. Inside a tile, quarter h in {0,1,2,3} covers
+ * k_local 16h..16h+15; column j in [0,128) owns 16 bytes at h*2048 + j*16,
+ * byte b holding the code of k_local = 16h + b. Codes outside [0,K) x [0,N)
+ * are 0.
+ */
+static inline int code8(const int8_t* q8, int64_t N, int64_t k, int64_t n) {
+#if ORACLE_MUTANT == 16
+    return (int)(uint8_t)q8[k * N + n];  /* codes read as unsigned bytes */
+#else
+    return (int)q8[k * N + n];
+#endif
+}
+
+int64_t oracle_tiled_bytes_w8(int64_t K, int64_t N) {
+    return ((N + 127) / 128) * ((K + 63) / 64) * 8192;
+}
+
+void oracle_tile_w8(const int8_t* q8, int64_t K, int64_t N, uint8_t* wt) {
+    int64_t NT = (N + 127) / 128, KT = (K + 63) / 64;
+    memset(wt, 0, (size_t)(NT * KT * 8192));
+    for (int64_t nt = 0; nt < NT; ++nt)
+        for (int64_t kt = 0; kt < KT; ++kt) {
+            uint8_t* tile = wt + (nt * KT + kt) * 8192;
+            for (int h = 0; h < 4; ++h)
+                for (int j = 0; j < 128; ++j)
+                    for (int b = 0; b < 16; ++b) {
+#if ORACLE_MUTANT == 17
+                        int64_t k = kt * 64 + 16 * h + (15 - b); /* bytes in reverse order */
+#else
+                        int64_t k = kt * 64 + 16 * h + b;
+#endif
+                        int64_t n = nt * 128 + j;
+                        if (k < K && n < N) tile[h * 2048 + j * 16 + b] = (uint8_t)q8[k * N + n];
+                    }
+        }
+}
+
+/* Dequantise column n of the 8-bit codes: w[k] = q8[k, n] * s[floor(k/G), n], exactly in double. */
+static void dequant_column_w8(const int8_t* q8, const uint16_t* S, int64_t N, int64_t K, int64_t G,
+                              int64_t n, double* w) {
+    int64_t groups = (K + G - 1) / G;
+    for (int64_t k = 0; k < K; ++k) {
+        int64_t g = scale_row(k, G);
+        if (g >= groups) g = groups - 1;
+        w[k] = (double)code8(q8, N, k, n) * scale_at(S, groups, N, g, n);
+    }
+}
+
+int oracle_gemm_w8(const uint16_t* A, const int8_t* q8, const uint16_t* S, int64_t M, int64_t N, int64_t K,
+                   int64_t G, uint16_t* C, int nthreads) {
+    if (M < 0 || N < 0 || K <= 0 || G <= 0) return 1;
+    double* a = widen_rows(A, M, K);
+    if (!a) return 2;
+    int failed = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        double* w = (double*)malloc((size_t)K * sizeof(double));
+        if (!w) {
+            failed = 1;
+        } else {
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 16)
+#endif
+            for (int64_t n = 0; n < N; ++n) {
+                dequant_column_w8(q8, S, N, K, G, n, w);
+                for (int64_t m = 0; m < M; ++m) C[m * N + n] = dot_round(a + m * K, w, K);
+            }
+            free(w);
+        }
+    }
+    free(a);
+    return failed ? 2 : 0;
+}

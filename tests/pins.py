@@ -419,9 +419,108 @@ def pin_quantize_edges(o) -> bool:
     return bool(np.all(S_t.view(np.uint16) == 0)) and bool(np.all(wp_t == 0))
 
 
+# ----------------------------------------------------- 8-bit codes (W8A16)
+
+def decode_tiled_w8(wt: np.ndarray, K: int, N: int) -> np.ndarray:
+    """Read every 8-bit code back out of the W8 tiled layout by its position formula."""
+    KT = (K + 63) // 64
+    q = np.zeros((K, N), dtype=np.int8)
+    k = np.arange(K)[:, None]
+    n = np.arange(N)[None, :]
+    kl = k % 64
+    byte = ((n // 128) * KT + k // 64) * 8192 + (kl // 16) * 2048 + (n % 128) * 16 + kl % 16
+    q[:, :] = wt[byte].view(np.int8)
+    return q
+
+
+def pin_w8_tiled_positions(o) -> bool:
+    """A single 8-bit code lands at the byte its position formula gives, unchanged."""
+    K, N = 100, 200
+    for k, n, byte in _read_table("tiled_positions_w8.txt"):
+        q = np.zeros((K, N), dtype=np.int8)
+        q[int(k), int(n)] = -77
+        wt = o.tile_w8(q)
+        nz = np.nonzero(wt)[0]
+        if len(nz) != 1 or nz[0] != int(byte) or wt[nz[0]] != np.uint8(256 - 77):
+            return False
+    return len(o.tile_w8(np.zeros((K, N), dtype=np.int8))) == 4 * 8192
+
+
+def pin_w8_tiled_roundtrip(o) -> bool:
+    """Random 8-bit codes, ragged K and N: decoding the tiles by formula returns q, and the
+    padding past K and N is zero."""
+    g = np.random.Generator(np.random.PCG64(16))
+    q = g.integers(-128, 128, size=(72, 136), dtype=np.int8)
+    wt = o.tile_w8(q)
+    if len(wt) != o.tiled_bytes_w8(72, 136) or len(wt) != 2 * 2 * 8192:
+        return False
+    ones = o.tile_w8(np.full((72, 136), -1, dtype=np.int8))
+    return bool(np.array_equal(decode_tiled_w8(wt, 72, 136), q)) and int(np.count_nonzero(ones)) == 72 * 136
+
+
+def w8_case(M, K, N, G, seed):
+    c = workloads.dense8(M, K, N, G, seed)
+    return c.A, c.q, c.S
+
+
+def pin_w8_exact_small(o) -> bool:
+    """8-bit codes: bit-exact against the integer brute force on small ragged shapes, with
+    the extreme codes -128 and 127 present."""
+    for (M, K, N, G, seed) in [(3, 40, 9, 16, 1), (2, 65, 7, 13, 2), (4, 96, 16, 32, 3), (1, 7, 5, 3, 4)]:
+        A, q, S = w8_case(M, K, N, G, seed)
+        q = q.copy()
+        q[0, 0], q[-1, -1] = -128, 127
+        got = o.gemm_w8(A, q, S, K, G)
+        want = exact.gemm_exact(A, q, S, G)
+        if not np.array_equal(got.view(np.uint16), want.view(np.uint16)):
+            return False
+    return True
+
+
+def pin_w8_closed_form(o) -> bool:
+    """Constant 8-bit codes and scale: C[m, n] = fp16(q * s * sum_k A[m, k])."""
+    M, K, N, G = 3, 192, 6, 64
+    g = np.random.Generator(np.random.PCG64(19))
+    A = g.standard_normal((M, K), dtype=np.float32).astype(np.float16)
+    for qv, sv in [(-128, 0.0001220703125), (127, 0.00031), (-1, 0.019)]:
+        s16 = np.float16(sv)
+        q = np.full((K, N), qv, dtype=np.int8)
+        S = np.full((-(-K // G), N), s16, dtype=np.float16)
+        got = o.gemm_w8(A, q, S, K, G).view(np.uint16)
+        s_units = exact.half_to_units(int(np.array(s16).view(np.uint16)))
+        for m in range(M):
+            row_units = sum(exact.half_to_units(int(b)) for b in A[m].view(np.uint16))
+            want = exact.round_units_to_half(row_units * qv * s_units, -48)
+            if not np.all(got[m] == want):
+                return False
+    return True
+
+
+def pin_w8_one_hot(o) -> bool:
+    """q = -128 only at k = pi(n), s = 2^-7: each weight is -1, so C[m, n] = -A[m, pi(n)] exactly."""
+    M, K, N, G = 5, 130, 12, 64
+    g = np.random.Generator(np.random.PCG64(20))
+    A = g.standard_normal((M, K), dtype=np.float32).astype(np.float16)
+    pi = np.array([0, 1, 15, 16, 63, 64, 65, 127, 128, 129, 77, 30])
+    q = np.zeros((K, N), dtype=np.int8)
+    q[pi, np.arange(N)] = -128
+    S = np.full((-(-K // G), N), 2.0 ** -7, dtype=np.float16)
+    got = o.gemm_w8(A, q, S, K, G)
+    return bool(np.array_equal(got.view(np.uint16), (-A[:, pi]).view(np.uint16)))
+
+
+def pin_w8_numpy_blas(o) -> bool:
+    """numpy float64 matmul of the dequantised 8-bit weights, rounded to fp16, agrees to 1 ulp."""
+    A, q, S = w8_case(6, 320, 48, 64, 22)
+    got = o.gemm_w8(A, q, S, 320, 64).view(np.uint16).astype(np.int32)
+    ref = (A.astype(np.float64) @ dequant_numpy(q, S, 64)).astype(np.float16)
+    return bool(np.all(np.abs(got - ref.view(np.uint16).astype(np.int32)) <= 1))
+
+
 PINS = [pin_half_widening, pin_half_rounding, pin_half_rounding_numpy, pin_pack_golden,
         pin_pack_all_bytes, pin_pack_random_odd_k, pin_tiled_positions, pin_tiled_roundtrip,
         pin_exact_small, pin_near_ties, pin_closed_form, pin_one_hot, pin_scale_duplication,
         pin_numpy_blas, pin_grouped_segments, pin_grouped_brute, pin_sample_matches_full,
         pin_quantize_golden, pin_quantize_properties, pin_quantize_scale_invariance,
-        pin_quantize_groups_independent, pin_quantize_edges]
+        pin_quantize_groups_independent, pin_quantize_edges, pin_w8_tiled_positions, pin_w8_tiled_roundtrip,
+        pin_w8_exact_small, pin_w8_closed_form, pin_w8_one_hot, pin_w8_numpy_blas]

@@ -40,6 +40,8 @@ MUTANTS = {
     13: "quantiser scale taken as max/8",
     14: "quantiser rounds halves to even",
     15: "quantiser scale from the whole column",
+    16: "8-bit codes read as unsigned",
+    17: "8-bit tiled layout with the bytes of a chunk reversed",
 }
 
 

@@ -106,6 +106,17 @@ def grouped(E: int, top_k: int, tokens: int, K: int, N: int, G: int, seed: int,
                        order.astype(np.int64), np.ascontiguousarray(A), offsets, q, S)
 
 
+def dense8(M: int, K: int, N: int, G: int, seed: int, name: str = "dense8") -> DenseCase:
+    """A W8A16 case: activations as in `dense`, signed 8-bit codes uniform over
+    [-128, 127], scales uniform over [S_LOW, S_HIGH] / 16, so that the weights q*s
+    span about the same range as the int4 cases'."""
+    g = _rng(seed)
+    A = g.standard_normal((M, K), dtype=np.float32).astype(np.float16)
+    q = g.integers(-128, 128, size=(K, N), dtype=np.int8)
+    S = (g.uniform(S_LOW, S_HIGH, size=(n_groups(K, G), N)) / 16).astype(np.float32).astype(np.float16)
+    return DenseCase(name, M, K, N, G, seed, A, q, S)
+
+
 @dataclasses.dataclass
 class MoeCase:
     name: str
