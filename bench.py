@@ -55,6 +55,11 @@ def algorithmic_bytes(M, N, K, G):
     return (K * N) // 2 + (-(-K // G)) * N * 2 + M * K * 2 + M * N * 2
 
 
+def algorithmic_bytes_w8(M, N, K, G):
+    """8-bit codes + fp16 scales + fp16 activations + fp16 output, each moved once."""
+    return K * N + (-(-K // G)) * N * 2 + M * K * 2 + M * N * 2
+
+
 def flops(M, N, K):
     return 2 * M * N * K
 
@@ -160,6 +165,24 @@ def job_throughput(units_per_rank: float, world: int, seconds_max: float) -> flo
     return world * units_per_rank / seconds_max
 
 
+def replay_stats(graph, launches_per_replay, reps):
+    """Per-launch device time of `reps` timed replays of a captured graph (CUDA events on
+    the replaying stream, one pair per replay): median, p10, p90 and mean, microseconds."""
+    import torch
+    samples = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(reps):
+        e0.record()
+        graph.replay()
+        e1.record()
+        e1.synchronize()
+        samples.append(e0.elapsed_time(e1) * 1e3 / launches_per_replay)
+    samples.sort()
+    q = lambda f: samples[min(len(samples) - 1, int(f * len(samples)))]
+    return {"median": round(statistics.median(samples), 3), "p10": round(q(0.10), 3), "p90": round(q(0.90), 3),
+            "mean": round(sum(samples) / len(samples), 3), "reps": reps, "launches_per_rep": launches_per_replay}
+
+
 SKINNY_SOURCES = ("w4a16_skinny.cu", "dequant.cuh", "ptx.cuh")
 
 
@@ -200,24 +223,55 @@ def sample_bytes(cols):
     return sum(algorithmic_bytes(m, cols, K_DIM, G_DIM) for m in M_STEP)
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(budget_s=12.0):
+    """The oracle on the host cores: the full decode step on all cores (the value), and a
+    column sample of it on one core (scaled to the step), each the median of a few runs."""
     import oracle
     o = oracle.load()
     case = workloads.dense(16, K_DIM, N_DIM, G_DIM, seed=1)
     wp = o.pack(case.q)
-    times = []
-    t_end = time.perf_counter() + budget_s
-    while True:
-        t0 = time.perf_counter()
+
+    def timed(step, budget, cap):
+        times = []
+        t_end = time.perf_counter() + budget
+        while True:
+            t0 = time.perf_counter()
+            step()
+            times.append(time.perf_counter() - t0)
+            if time.perf_counter() > t_end or len(times) >= cap:
+                break
+        return statistics.median(times), len(times)
+
+    def full_step():
         for m in M_STEP:
             o.gemm(case.A[:m], wp, case.S, K_DIM, G_DIM)
-        times.append(time.perf_counter() - t0)
-        if time.perf_counter() > t_end or len(times) >= 20:
-            break
-    t = statistics.median(times)
-    return {"value": step_bytes() / t / 1e9, "unit": "GB/s", "cores": o.threads(), "kind": "oracle",
-            "sample": f"full decode step (M=1 and M=16, K=N=4096, G=128), median of {len(times)} runs, "
-                      f"{t * 1e3:.1f} ms per step"}
+    t_all, n_all = timed(full_step, budget_s, 20)
+    cols = 512
+    wp1, S1 = oracle_sample(o, case, cols)
+
+    def one_core_step():
+        for m in M_STEP:
+            o.gemm(case.A[:m], wp1, S1, K_DIM, G_DIM, threads=1)
+    t_one, n_one = timed(one_core_step, budget_s / 2, 5)
+    one_value = sample_bytes(cols) / t_one / 1e9
+    return {"value": step_bytes() / t_all / 1e9, "unit": "GB/s", "cores": o.threads(), "kind": "oracle",
+            "sample": f"full decode step (M=1 and M=16, K=N=4096, G=128), median of {n_all} runs, "
+                      f"{t_all * 1e3:.1f} ms per step",
+            "one_core": {"value": one_value, "unit": "GB/s", "cores": 1,
+                         "sample": f"M=1 and M=16 over the first {cols} of {N_DIM} columns, median of {n_one} "
+                                   f"runs, {t_one * 1e3:.1f} ms"},
+            "affinity_cores": len(os.sched_getaffinity(0)), "cpu_model": cpu_model()}
 
 
 # ------------------------------------------------------------------ our arm
@@ -307,6 +361,14 @@ def run_ours(args):
     value = job_throughput(K * step_bytes(), world, sec) / 1e9
     tflops = job_throughput(K * step_flops(), world, sec) / 1e12
 
+    # Distribution of the step time: 100 timed replays of a 20-step graph (after the timed region).
+    g_stats = capture(20, 7)
+    for _ in range(3):
+        g_stats.replay()
+    torch.cuda.synchronize()
+    step_stats = replay_stats(g_stats, 20, 100)
+    del g_stats
+
     status = w4.device_status(clear=True)
     if status != w4.OK:
         raise RuntimeError(f"device status after the timed region: {w4.status_string(status)}")
@@ -322,28 +384,51 @@ def run_ours(args):
     C1_d, C16_d = C_d[:1], C_d[1:]
     K_e2e = min(K, 2000)
 
+    # The step as a decode loop runs it: the host->device copy of the step's
+    # activations, the two GEMMs through the C entry point, the device->host copy
+    # of their results, recorded once into a CUDA graph of E2E_GRAPH_STEPS steps
+    # (rotating weight copies as in the timed region) and replayed; every step
+    # still moves its inputs in and its outputs out.
+    E2E_GRAPH_STEPS = 16
+    cgemm = w4.load().w4a16_gemm
+    a1, a16, c1, c16 = A1_d.data_ptr(), A16_d.data_ptr(), C1_d.data_ptr(), C16_d.data_ptr()
+    wptr = [x.data_ptr() for x in wts]
+    sptr = [x.data_ptr() for x in Ss]
+
     def e2e_step(i):
-        A_d.copy_(A_h, non_blocking=True)
+        st = torch.cuda.current_stream(dev).cuda_stream
         r1, r2 = (2 * i) % R, (2 * i + 1) % R
-        w4.gemm(A1_d, wts[r1], Ss[r1], N_DIM, G_DIM, out=C1_d)
-        w4.gemm(A16_d, wts[r2], Ss[r2], N_DIM, G_DIM, out=C16_d)
+        A_d.copy_(A_h, non_blocking=True)
+        if cgemm(a1, wptr[r1], sptr[r1], c1, 1, N_DIM, K_DIM, G_DIM, st) or \
+                cgemm(a16, wptr[r2], sptr[r2], c16, 16, N_DIM, K_DIM, G_DIM, st):
+            raise RuntimeError("a GEMM call failed in the end-to-end loop")
         C_h.copy_(C_d, non_blocking=True)
 
-    for i in range(20):
+    for i in range(E2E_GRAPH_STEPS):
         e2e_step(i)
+    torch.cuda.synchronize()
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e):
+        for i in range(E2E_GRAPH_STEPS):
+            e2e_step(i)
+    reps_e2e = max(1, K_e2e // E2E_GRAPH_STEPS)
+    K_e2e = reps_e2e * E2E_GRAPH_STEPS
+    for _ in range(3):
+        g_e2e.replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record()
-    for i in range(K_e2e):
-        e2e_step(i)
+    for _ in range(reps_e2e):
+        g_e2e.replay()
     f1.record()
     f1.synchronize()
     e2e_sec = max_over_ranks(f0.elapsed_time(f1), dev) / 1e3
     e2e = {"value": job_throughput(K_e2e * step_bytes(), world, e2e_sec) / 1e9, "unit": "GB/s",
            "h2d_bytes_per_step": sum(m * K_DIM * 2 for m in M_STEP),
-           "d2h_bytes_per_step": sum(m * N_DIM * 2 for m in M_STEP), "steps": K_e2e}
+           "d2h_bytes_per_step": sum(m * N_DIM * 2 for m in M_STEP), "steps": K_e2e,
+           "launch": f"CUDA graph of {E2E_GRAPH_STEPS} steps (copy in, two w4a16_gemm calls, copy out), replayed"}
 
     extra = per_config(w4, dev) if (rank == 0 and not args.no_configs) else None
     peaks = load_peaks()
@@ -363,6 +448,8 @@ def run_ours(args):
                      "peak_source": f"{peaks['source']} (copy bandwidth)",
                      "kernel": "w4a16_skinny_kernel (M <= 16: 8- or 16-row token tiles, K split over a cluster)"},
         "e2e": e2e,
+        "step_us": dict(step_stats, note="device time per step (one M=1 and one M=16 launch), 100 CUDA-graph "
+                                         "replays of 20 steps, after the timed region"),
         "gpu_launches": world * 2 * K,
         "launch": {f"M={m}": w4.w4a16_gemm_launch_info(m, N_DIM, K_DIM, G_DIM)[1].as_dict() for m in M_STEP},
         "clocks": clocks,
@@ -405,6 +492,52 @@ def per_config(w4, dev):
                     raise RuntimeError(w4.status_string(rc))
             fl = flops(M, N, K)
             by = algorithmic_bytes(M, N, K, G)
+        elif cfg["kind"] == "dense8":
+            wt = w4.repack_w8(torch.from_numpy(c.q).to(dev))
+            S = torch.from_numpy(c.S).to(dev)
+            A = torch.from_numpy(c.A).to(dev)
+            C = torch.empty((c.M, c.N), dtype=torch.float16, device=dev)
+            per = wt.numel() + S.numel() * 2 + A.numel() * 2 + C.numel() * 2
+            R = max(2, math.ceil(2 * l2 / per) + 1)
+            bufs = [(wt, S, A, C)] + [(wt.clone(), S.clone(), A.clone(), torch.empty_like(C)) for _ in range(R - 1)]
+            M, N, K, G = c.M, c.N, c.K, c.G
+
+            def launch(r, b=bufs, M=M, N=N, K=K, G=G):
+                wt_, S_, A_, C_ = b[r]
+                rc = w4.w8a16_gemm(A_, wt_, S_, C_, M, N, K, G)
+                if rc:
+                    raise RuntimeError(w4.status_string(rc))
+            fl = flops(M, N, K)
+            by = algorithmic_bytes_w8(M, N, K, G)
+        elif cfg["kind"] == "moe":
+            # The whole expert layer: route, dispatch, gather, up (GELU epilogue), down, combine.
+            def expert_set(q, S):
+                return ([w4.prepare_weights(torch.from_numpy(q[e]).to(dev))[1] for e in range(c.E)],
+                        [torch.from_numpy(S[e]).to(dev) for e in range(c.E)])
+            up, down = expert_set(c.q_up, c.S_up), expert_set(c.q_down, c.S_down)
+            X = torch.from_numpy(c.X).to(dev)
+            lg = torch.from_numpy(c.logits).to(dev)
+            C = torch.empty((c.tokens, c.H), dtype=torch.float16, device=dev)
+            ws = torch.empty(w4.w4a16_moe_workspace_size(c.tokens, c.E, c.top_k, c.H, c.I), dtype=torch.uint8,
+                             device=dev)
+            per = sum(x.numel() for x in up[0] + down[0]) + sum(x.numel() * 2 for x in up[1] + down[1])
+            R = max(2, math.ceil(2 * l2 / per) + 1)
+            sets = [(up, down)] + [(([x.clone() for x in up[0]], [x.clone() for x in up[1]]),
+                                    ([x.clone() for x in down[0]], [x.clone() for x in down[1]]))
+                                   for _ in range(R - 1)]
+
+            def launch(r, sets=sets, X=X, lg=lg, C=C, ws=ws, c=c):
+                (wu, su), (wd, sd) = sets[r]
+                rc = w4.w4a16_moe_layer(X, lg, wu, su, wd, sd, C, c.tokens, c.E, c.top_k, c.H, c.I, c.G,
+                                        w4.ACT_GELU_ERF, ws, ws.numel())
+                if rc:
+                    raise RuntimeError(w4.status_string(rc))
+            rows = c.tokens * c.top_k
+            fl = 2 * flops(rows, c.I, c.H)
+            # both projections' weights and scales, activations in and out of each, the
+            # gather and the combine; every expert receives rows at this size
+            by = c.E * (algorithmic_bytes(0, c.I, c.H, c.G) + algorithmic_bytes(0, c.H, c.I, c.G)) + \
+                rows * (c.H + c.I) * 2 * 2 + (c.tokens * c.H * 2) * 2 + rows * c.H * 2 * 2
         else:
             wts = [w4.prepare_weights(torch.from_numpy(c.q[e]).to(dev))[1] for e in range(c.E)]
             Ss = [torch.from_numpy(c.S[e]).to(dev) for e in range(c.E)]
@@ -424,26 +557,25 @@ def per_config(w4, dev):
             by = sum(algorithmic_bytes(int(c.offsets[e + 1] - c.offsets[e]), c.N, c.K, c.G) for e in range(c.E))
         launch(0)
         torch.cuda.synchronize()
-        n = 200 if fl < 1e10 else 40
+        n = 20 if fl < 1e10 else 4
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for i in range(n):
                 launch(i % R)
-        g.replay()
+        for _ in range(3):
+            g.replay()
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        g.replay()
-        e1.record()
-        e1.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / n
+        st = replay_stats(g, n, 100)
+        us = st["median"]
         gbs = by / (us * 1e-6) / 1e9
         tf = fl / (us * 1e-6) / 1e12
         t_roof = max(by / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
-        out[name] = {"us_per_launch": round(us, 3), "GB/s": round(gbs, 1), "TFLOP/s": round(tf, 2),
+        out[name] = {"us_per_launch": round(us, 3), "us_p10": st["p10"], "us_p90": st["p90"],
+                     "GB/s": round(gbs, 1), "TFLOP/s": round(tf, 2),
                      "roofline_frac": round(t_roof / (us * 1e-6), 4),
                      "bound": "hbm" if by / (peaks["hbm_gbs"] * 1e9) >= fl / (peaks["bf16_tflops"] * 1e12)
-                     else "tensor", "rotating_copies": R}
+                     else "tensor", "rotating_copies": R, "timing": f"median of {st['reps']} CUDA-graph replays of "
+                                                                  f"{n} launches each"}
         del g
     out["quantize"] = quantize_timing(w4, dev, peaks, l2)
     status = w4.device_status(clear=True)
@@ -473,21 +605,19 @@ def quantize_timing(w4, dev, peaks, l2, K=4096, N=14336, G=128):
             raise RuntimeError(w4.status_string(rc))
     launch(0)
     torch.cuda.synchronize()
-    n = 40
+    n = 4
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(n):
             launch(i % R)
-    g.replay()
+    for _ in range(3):
+        g.replay()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    g.replay()
-    e1.record()
-    e1.synchronize()
-    us = e0.elapsed_time(e1) * 1e3 / n
+    st = replay_stats(g, n, 100)
+    us = st["median"]
     del g
-    return {"us_per_launch": round(us, 3), "GB/s": round(by / (us * 1e-6) / 1e9, 1),
+    return {"us_per_launch": round(us, 3), "us_p10": st["p10"], "us_p90": st["p90"],
+            "GB/s": round(by / (us * 1e-6) / 1e9, 1),
             "roofline_frac": round(by / (peaks["hbm_gbs"] * 1e9) / (us * 1e-6), 4), "bound": "hbm",
             "rotating_copies": R, "shape": {"K": K, "N": N, "G": G}}
 

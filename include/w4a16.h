@@ -63,8 +63,28 @@ enum {
     W4A16_ERR_UNSUPPORTED = 3,  /* shape outside the GPU contract, or no sm_100 device */
     W4A16_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
     W4A16_ERR_TIMEOUT = 5,      /* device status: a bounded wait inside a kernel ran out */
-    W4A16_ERR_BAD_OFFSETS = 6   /* device status: expert offsets not 0 = o[0] <= ... <= o[E] = rows */
+    W4A16_ERR_BAD_OFFSETS = 6,  /* device status: expert offsets not 0 = o[0] <= ... <= o[E] = rows */
+    W4A16_ERR_BAD_ROUTING = 7   /* device status: an expert id out of range or repeated within a token,
+                                   or a gathered-row index out of range */
 };
+
+/* Elementwise activations of the expert layer (Int4 Moe Plugin page,
+ * constructor parameter activationType), applied to the fp16 result x of the
+ * up projection and rounded to fp16 again:
+ *   IDENTITY   x
+ *   RELU       max(x, 0)
+ *   GELU_ERF   x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2))
+ *   GELU_TANH  0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
+ * evaluated in fp32 on the device. */
+enum {
+    W4A16_ACT_IDENTITY = 0,
+    W4A16_ACT_RELU = 1,
+    W4A16_ACT_GELU_ERF = 2,
+    W4A16_ACT_GELU_TANH = 3
+};
+
+/* Largest topK the expert layer accepts. */
+#define W4A16_MAX_TOPK 8
 
 /* Largest number of experts one w4a16_grouped_gemm call accepts. */
 #define W4A16_MAX_EXPERTS 64
@@ -133,6 +153,90 @@ int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const* Wt, const 
                        const int32_t* offsets_dev, w4a16_half* C_dev, int64_t E, int64_t total_rows,
                        int64_t N, int64_t K, int64_t G, void* stream);
 
+/* w4a16_grouped_gemm with the activation `act` (W4A16_ACT_*) applied to each
+ * fp16 result element in the epilogue: C = fp16(act(fp16(A x dequant(W)))).
+ * The expert layer's up projection (Int4 Moe Plugin page: hiddenSize ->
+ * moeInterSize, then activationType). Same contract and errors as
+ * w4a16_grouped_gemm; INVALID_ARG also for an unknown act. */
+int w4a16_grouped_gemm_act(const w4a16_half* A_dev, const uint8_t* const* Wt, const w4a16_half* const* S,
+                           const int32_t* offsets_dev, w4a16_half* C_dev, int64_t E, int64_t total_rows,
+                           int64_t N, int64_t K, int64_t G, int act, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * The INT4 mixture-of-experts layer (Int4 Moe Plugin page: constructor
+ * parameters numExperts E, topK k, hiddenSize H, moeInterSize I,
+ * activationType, quantizationGroupSize G; getWorkspaceSize; enqueue with a
+ * workspace and a stream; one output). The page names the parameters, not the
+ * steps; the steps are the plain reading of them, for T tokens:
+ *
+ *   1. route     ids[t, 0..k-1]: the k experts with the largest router logits
+ *                (ties: the lower expert index first), in descending order;
+ *                weights[t, j] = softmax over the k selected logits (fp32).
+ *   2. dispatch  the T*k (token, slot) pairs grouped by expert, stable in the
+ *                flat order t*k + j: offsets[E+1] (expert e owns gathered rows
+ *                offsets[e] .. offsets[e+1]-1), pos[t, j] (the gathered row of
+ *                the pair), src_row[r] (the token of gathered row r).
+ *   3. gather    Xg[r] = X[src_row[r]].
+ *   4. up        A = fp16(act(fp16(Xg x dequant(W_up[e])))), per expert [H -> I].
+ *   5. down      Y = fp16(A x dequant(W_down[e])), per expert [I -> H].
+ *   6. combine   out[t] = fp16(sum over j of weights[t, j] * Y[pos[t, j]]),
+ *                fp32 arithmetic in slot order.
+ *
+ * Each step is an entry point of its own; w4a16_moe_layer enqueues all six on
+ * one stream with intermediates in a caller-owned workspace. Sizes: 1 <= E <=
+ * W4A16_MAX_EXPERTS, 1 <= k <= min(E, W4A16_MAX_TOPK), T*k < 2^31. Router
+ * logits must be finite (a NaN logit is never preferred over a finite one, so
+ * the ids stay valid, but its weight is NaN).
+ * ------------------------------------------------------------------------- */
+
+/* Step 1. logits_dev [T, E] fp16 -> ids_dev [T, k] int32, weights_dev [T, k]
+ * fp32. T == 0 is a no-op. Errors: INVALID_ARG, UNSUPPORTED (no sm_100
+ * device), CUDA. */
+int w4a16_moe_route(const w4a16_half* logits_dev, int32_t* ids_dev, float* weights_dev, int64_t T, int64_t E,
+                    int64_t top_k, void* stream);
+
+/* Step 2. ids_dev [T, k] int32 -> offsets_dev [E+1], pos_dev [T, k],
+ * src_row_dev [T*k] (all int32). If any id is outside [0, E) or repeated
+ * within a token, the kernel writes offsets all 0, pos and src_row all -1, and
+ * latches W4A16_ERR_BAD_ROUTING. T == 0 writes offsets all 0. Errors:
+ * INVALID_ARG, UNSUPPORTED, CUDA. */
+int w4a16_moe_dispatch(const int32_t* ids_dev, int32_t* offsets_dev, int32_t* pos_dev, int32_t* src_row_dev,
+                       int64_t T, int64_t E, int64_t top_k, void* stream);
+
+/* Step 3. X_dev [T, H] -> Xg_dev [rows, H] with Xg[r] = X[src_row[r]]. H % 8
+ * == 0; X_dev and Xg_dev 16-byte aligned. A row index outside [0, T) writes
+ * zeros and latches W4A16_ERR_BAD_ROUTING. Errors: INVALID_ARG, MISALIGNED,
+ * UNSUPPORTED, CUDA. */
+int w4a16_moe_gather(const w4a16_half* X_dev, const int32_t* src_row_dev, w4a16_half* Xg_dev, int64_t T,
+                     int64_t rows, int64_t H, void* stream);
+
+/* Step 6. Y_dev [T*k, H], weights_dev [T, k] fp32, pos_dev [T, k] -> out_dev
+ * [T, H]. H % 8 == 0; Y_dev and out_dev 16-byte aligned. A term whose pos is
+ * outside [0, T*k) is left out and W4A16_ERR_BAD_ROUTING latched. Errors:
+ * INVALID_ARG, MISALIGNED, UNSUPPORTED, CUDA. */
+int w4a16_moe_combine(const w4a16_half* Y_dev, const float* weights_dev, const int32_t* pos_dev,
+                      w4a16_half* out_dev, int64_t T, int64_t top_k, int64_t H, void* stream);
+
+/* Bytes of workspace w4a16_moe_layer needs (the page's getWorkspaceSize):
+ * ids, weights, pos, src_row, offsets, the gathered rows [T*k, H], the
+ * activated up projection [T*k, I] and the down projection [T*k, H], each
+ * starting on a 256-byte boundary. Returns -1 for invalid sizes. */
+int64_t w4a16_moe_workspace_size(int64_t T, int64_t E, int64_t top_k, int64_t H, int64_t I);
+
+/* The whole layer: out_dev [T, H] from hidden states X_dev [T, H] and router
+ * logits logits_dev [T, E]. Wt_up / S_up / Wt_down / S_down are HOST arrays of
+ * E device pointers: tiled weights [H -> I] and [I -> H] with scales
+ * [ceil(H/G), I] and [ceil(I/G), H]. workspace_dev (16-byte aligned, at least
+ * w4a16_moe_workspace_size bytes) is caller-owned; nothing in it needs to be
+ * initialised, and two calls that overlap on the GPU must not share it.
+ * Contract of the GEMMs (H, I multiples of 8, G % 16 == 0). T == 0 is a no-op.
+ * Errors: INVALID_ARG (also workspace too small or unknown act), MISALIGNED,
+ * UNSUPPORTED, CUDA. */
+int w4a16_moe_layer(const w4a16_half* X_dev, const w4a16_half* logits_dev, const uint8_t* const* Wt_up,
+                    const w4a16_half* const* S_up, const uint8_t* const* Wt_down, const w4a16_half* const* S_down,
+                    w4a16_half* out_dev, int64_t T, int64_t E, int64_t top_k, int64_t H, int64_t I, int64_t G,
+                    int act, void* workspace_dev, int64_t workspace_bytes, void* stream);
+
 /* Declares (enable != 0) or withdraws (enable == 0) the promise that no
  * kernel on the calling streams writes the tiled weights or the scales passed
  * to w4a16_gemm right before that call, i.e. the weights are static (prepared
@@ -161,6 +265,90 @@ typedef struct {
 int w4a16_gemm_launch_info(int64_t M, int64_t N, int64_t K, int64_t G, w4a16_launch_info* info);
 int w4a16_grouped_launch_info(int64_t E, int64_t total_rows, int64_t N, int64_t K, int64_t G,
                               w4a16_launch_info* info);
+
+/* ---------------------------------------------------------------------------
+ * W8A16: the INT8 weight-only variant (the FP8-vs-INT8 TensorRT-LLM comparison
+ * page lists INT8 weight-only with an FP16 KV cache among its INT8
+ * configurations). The same group-wise product with signed 8-bit codes:
+ *     C[m, n] = fp16( sum_k A[m, k] * q8[k, n] * s[floor(k / G), n] ),
+ * q8 in [-128, 127], s [ceil(K/G), N] fp16. Canonical codes are int8 [K, N]
+ * row-major, one per byte (no packing). Tiled layout (the GEMM's operand),
+ * w8a16_tiled_bytes(K, N) bytes: ceil(N/128) x ceil(K/64) tiles of 8192 bytes,
+ * tile (nt, kt) at byte (nt*ceil(K/64)+kt)*8192; inside a tile, quarter h
+ * (k_local 16h..16h+15) of column j is 16 bytes at h*2048 + j*16, byte b
+ * holding k_local 16h + b as a two's-complement byte; rows k >= K and columns
+ * n >= N hold 0. The product runs on the tensor-core kernel for every M.
+ * ------------------------------------------------------------------------- */
+
+/* Size in bytes of the 8-bit tiled layout for K x N codes (0 if K or N <= 0). */
+int64_t w8a16_tiled_bytes(int64_t K, int64_t N);
+
+/* One-off repack of int8 codes q_dev [K, N] into the 8-bit tiled layout wt_dev
+ * (16-byte aligned). Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED (no sm_100
+ * device), CUDA. */
+int w8a16_repack(const int8_t* q_dev, uint8_t* wt_dev, int64_t K, int64_t N, void* stream);
+
+/* C_dev [M, N] = A_dev [M, K] x (q8 * s) from the 8-bit tiled layout Wt8_dev and
+ * scales S_dev [ceil(K/G), N]. Same GPU contract, rounding and errors as
+ * w4a16_gemm (each dequantised weight q*s rounded to fp16 before the product,
+ * fp32 accumulation, one rounding of the result). */
+int w8a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt8_dev, const w4a16_half* S_dev, w4a16_half* C_dev,
+               int64_t M, int64_t N, int64_t K, int64_t G, void* stream);
+
+/* How w8a16_gemm will launch for a shape (no work is enqueued). */
+int w8a16_gemm_launch_info(int64_t M, int64_t N, int64_t K, int64_t G, w4a16_launch_info* info);
+
+/* ---------------------------------------------------------------------------
+ * Tactics (Int4GroupwiseGemmPluginV2 page: getNbTactics / getValidTactics list
+ * the valid variants as ids >= 1, setTactic selects one, 0 is the default
+ * variant; configurePlugin captures the optimum M the tuning is done for; the
+ * timing cache tunes identical shapes once). A tactic of w4a16_gemm for a
+ * shape (M, N, K, G) is one launch form: the skinny kernel (M <= 16 only) with
+ * a K split over 1..8 cluster CTAs, one or two K halves per CTA and a ring
+ * depth, or the tensor-core kernel with a token tile of 16..256 rows and a K
+ * split of 1, 2, 4 or 8. Every tactic computes the same product (the K split
+ * changes the fp32 summation order only). The process-wide table maps a shape
+ * on a device to its tactic; w4a16_gemm and w4a16_gemm_launch_info use the
+ * table's tactic when it holds one for the exact shape, else the built-in
+ * heuristic. The table is guarded by a mutex; its lookup is skipped while it
+ * is empty.
+ * ------------------------------------------------------------------------- */
+
+/* The ids (1..count) of the valid tactics for a shape, skinny forms first.
+ * Writes min(count, capacity) ids to `tactics` and the total to *count.
+ * Errors: INVALID_ARG, UNSUPPORTED (shape outside the GPU contract). */
+int w4a16_get_valid_tactics(int64_t M, int64_t N, int64_t K, int64_t G, int32_t* tactics, int32_t capacity,
+                            int32_t* count);
+
+/* The launch form of one tactic id for a shape. Errors: INVALID_ARG (also an
+ * id outside 1..count), UNSUPPORTED. */
+int w4a16_tactic_launch_info(int64_t M, int64_t N, int64_t K, int64_t G, int32_t tactic,
+                             w4a16_launch_info* info);
+
+/* Pins tactic `tactic` for the shape on the current device (0 removes the
+ * entry: the heuristic applies again). Errors: INVALID_ARG, UNSUPPORTED. */
+int w4a16_set_tactic(int64_t M, int64_t N, int64_t K, int64_t G, int32_t tactic);
+
+/* The table's tactic for the shape on the current device (0 if none). */
+int w4a16_get_tactic(int64_t M, int64_t N, int64_t K, int64_t G, int32_t* tactic);
+
+/* Empties the tactic table. Always W4A16_OK. */
+int w4a16_clear_tactics(void);
+
+/* Times every valid tactic for the shape on the caller's buffers (A, Wt, S
+ * read; C overwritten) on `stream`, `reps` launches each after one untimed
+ * launch, and stores the fastest in the table (the page's timing cache).
+ * With flush_dev (flush_bytes > 0; a device buffer larger than the L2 cache,
+ * overwritten) every timed launch starts after the buffer is rewritten, so the
+ * weights come from HBM as they do when many layers' weights stream by; with
+ * flush_dev NULL the launches run back to back. Blocks the host until the
+ * timing is done: call it at setup, not while the stream is being captured.
+ * Writes the winning id to *best_tactic and its mean time per launch in
+ * microseconds to *best_us (if not NULL). Same contract and errors as
+ * w4a16_gemm, INVALID_ARG also for reps outside 1..10000. */
+int w4a16_autotune(const w4a16_half* A_dev, const uint8_t* Wt_dev, const w4a16_half* S_dev, w4a16_half* C_dev,
+                   int64_t M, int64_t N, int64_t K, int64_t G, int32_t reps, void* flush_dev,
+                   int64_t flush_bytes, int32_t* best_tactic, float* best_us, void* stream);
 
 /* Test aid for the failure path of the bounded device waits (no counterpart
  * on the plugin pages). For every later launch of the tensor-core GEMM kernel

@@ -1,0 +1,58 @@
+"""W8A16 (8-bit codes) on the GPU against the oracle: the repack into the 8-bit
+tiled layout bit for bit, and the product element by element within the GEMM
+tolerance 1e-2 + 5e-3 |ref|, on ragged shapes, every group size form, decode
+and prefill sizes."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import weight_only_int4_wise_b200 as w
+from gpu_util import dev, guarded_output, guards_intact, within_tolerance
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def o():
+    return oracle.load()
+
+
+@pytest.mark.parametrize("K,N", [(64, 128), (72, 136), (130, 200), (4096, 264)])
+def test_repack_w8_bit_exact(o, K, N):
+    q = np.random.Generator(np.random.PCG64(K + N)).integers(-128, 128, size=(K, N), dtype=np.int8)
+    wt = w.repack_w8(dev(q))
+    torch.cuda.synchronize()
+    assert np.array_equal(wt.cpu().numpy(), o.tile_w8(q))
+
+
+def run_w8(o, c):
+    wt = w.repack_w8(dev(c.q))
+    A, S = dev(c.A), dev(c.S)
+    flat, C, pad = guarded_output(c.M, c.N)
+    assert w.w8a16_gemm(A, wt, S, C, c.M, c.N, c.K, c.G) == w.OK
+    torch.cuda.synchronize()
+    got = C.cpu().numpy()
+    ref = o.gemm_w8(c.A, c.q, c.S, c.K, c.G)
+    ok, err, rel = within_tolerance(got, ref)
+    assert ok, f"W8 {c.M}x{c.K}x{c.N} G={c.G}: max abs err {err}, max rel err {rel}"
+    assert guards_intact(flat, pad, c.M * c.N)
+    assert w.device_status() == w.OK
+
+
+@pytest.mark.parametrize("M,K,N,G", [
+    (1, 4096, 4096, 128),    # decode: one 16-row token tile, K split over a cluster
+    (16, 1024, 512, 64),
+    (5, 136, 264, 32),       # per-word scales (G not a multiple of 64), ragged column tile
+    (40, 1024, 512, 48),     # groups straddling the 64-deep stages
+    (300, 512, 392, 128),    # several token tiles
+    (33, 4096, 256, 8192),   # G > K: one group
+])
+def test_w8_gemm_matches_oracle(o, M, K, N, G):
+    run_w8(o, workloads.dense8(M, K, N, G, seed=M * 3 + N))
+
+
+@pytest.mark.parametrize("name", ["w8_decode_m16", "w8_prefill"])
+def test_w8_full_size(o, name):
+    run_w8(o, workloads.make(name))

@@ -23,12 +23,22 @@ ERR_UNSUPPORTED = 3
 ERR_CUDA = 4
 ERR_TIMEOUT = 5
 ERR_BAD_OFFSETS = 6
+ERR_BAD_ROUTING = 7
 MAX_EXPERTS = 64
+MAX_TOPK = 8
+ACT_IDENTITY = 0
+ACT_RELU = 1
+ACT_GELU_ERF = 2
+ACT_GELU_TANH = 3
 
 EXPORTED = [
     "w4a16_status_string", "w4a16_pack", "w4a16_unpack", "w4a16_tiled_bytes", "w4a16_repack",
     "w4a16_gemm", "w4a16_grouped_gemm", "w4a16_gemm_launch_info", "w4a16_grouped_launch_info",
     "w4a16_device_status", "w4a16_set_static_weights", "w4a16_quantize", "w4a16_set_fault_injection",
+    "w4a16_grouped_gemm_act", "w4a16_moe_route", "w4a16_moe_dispatch", "w4a16_moe_gather", "w4a16_moe_combine",
+    "w4a16_moe_workspace_size", "w4a16_moe_layer", "w4a16_get_valid_tactics", "w4a16_tactic_launch_info",
+    "w4a16_set_tactic", "w4a16_get_tactic", "w4a16_clear_tactics", "w4a16_autotune",
+    "w8a16_tiled_bytes", "w8a16_repack", "w8a16_gemm", "w8a16_gemm_launch_info",
 ]
 
 
@@ -85,6 +95,45 @@ def load() -> ctypes.CDLL:
         lib.w4a16_set_static_weights.restype = ctypes.c_int
         lib.w4a16_set_fault_injection.argtypes = [_i64, _i64]
         lib.w4a16_set_fault_injection.restype = ctypes.c_int
+        lib.w4a16_grouped_gemm_act.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _vp, _i64,
+                                               _i64, _i64, _i64, _i64, ctypes.c_int, _vp]
+        lib.w4a16_grouped_gemm_act.restype = ctypes.c_int
+        lib.w4a16_moe_route.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp]
+        lib.w4a16_moe_route.restype = ctypes.c_int
+        lib.w4a16_moe_dispatch.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
+        lib.w4a16_moe_dispatch.restype = ctypes.c_int
+        lib.w4a16_moe_gather.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp]
+        lib.w4a16_moe_gather.restype = ctypes.c_int
+        lib.w4a16_moe_combine.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
+        lib.w4a16_moe_combine.restype = ctypes.c_int
+        lib.w4a16_moe_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i64]
+        lib.w4a16_moe_workspace_size.restype = _i64
+        lib.w4a16_moe_layer.argtypes = [_vp, _vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                                        ctypes.POINTER(_vp), _vp, _i64, _i64, _i64, _i64, _i64, _i64, ctypes.c_int,
+                                        _vp, _i64, _vp]
+        lib.w4a16_moe_layer.restype = ctypes.c_int
+        lib.w8a16_tiled_bytes.argtypes = [_i64, _i64]
+        lib.w8a16_tiled_bytes.restype = _i64
+        lib.w8a16_repack.argtypes = [_vp, _vp, _i64, _i64, _vp]
+        lib.w8a16_repack.restype = ctypes.c_int
+        lib.w8a16_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]
+        lib.w8a16_gemm.restype = ctypes.c_int
+        lib.w8a16_gemm_launch_info.argtypes = [_i64, _i64, _i64, _i64, ctypes.POINTER(LaunchInfo)]
+        lib.w8a16_gemm_launch_info.restype = ctypes.c_int
+        _i32p = ctypes.POINTER(ctypes.c_int32)
+        lib.w4a16_get_valid_tactics.argtypes = [_i64, _i64, _i64, _i64, _i32p, ctypes.c_int32, _i32p]
+        lib.w4a16_get_valid_tactics.restype = ctypes.c_int
+        lib.w4a16_tactic_launch_info.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int32, ctypes.POINTER(LaunchInfo)]
+        lib.w4a16_tactic_launch_info.restype = ctypes.c_int
+        lib.w4a16_set_tactic.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int32]
+        lib.w4a16_set_tactic.restype = ctypes.c_int
+        lib.w4a16_get_tactic.argtypes = [_i64, _i64, _i64, _i64, _i32p]
+        lib.w4a16_get_tactic.restype = ctypes.c_int
+        lib.w4a16_clear_tactics.argtypes = []
+        lib.w4a16_clear_tactics.restype = ctypes.c_int
+        lib.w4a16_autotune.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.c_int32, _vp, _i64, _i32p,
+                                       ctypes.POINTER(ctypes.c_float), _vp]
+        lib.w4a16_autotune.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -158,6 +207,105 @@ def w4a16_grouped_gemm(A, Wt: Sequence, S: Sequence, offsets, C, E: int, total_r
     s_arr = (_vp * max(1, len(S)))(*[_addr(s) for s in S])
     return load().w4a16_grouped_gemm(_addr(A), wt_arr, s_arr, _addr(offsets), _addr(C), E, total_rows, N, K, G,
                                      _stream(stream))
+
+
+def _ptr_array(xs: Sequence):
+    return (_vp * max(1, len(xs)))(*[_addr(x) for x in xs])
+
+
+def w4a16_grouped_gemm_act(A, Wt: Sequence, S: Sequence, offsets, C, E: int, total_rows: int, N: int, K: int,
+                           G: int, act: int, stream=None) -> int:
+    return load().w4a16_grouped_gemm_act(_addr(A), _ptr_array(Wt), _ptr_array(S), _addr(offsets), _addr(C), E,
+                                         total_rows, N, K, G, act, _stream(stream))
+
+
+def w4a16_moe_route(logits, ids, weights, T: int, E: int, top_k: int, stream=None) -> int:
+    return load().w4a16_moe_route(_addr(logits), _addr(ids), _addr(weights), T, E, top_k, _stream(stream))
+
+
+def w4a16_moe_dispatch(ids, offsets, pos, src_row, T: int, E: int, top_k: int, stream=None) -> int:
+    return load().w4a16_moe_dispatch(_addr(ids), _addr(offsets), _addr(pos), _addr(src_row), T, E, top_k,
+                                     _stream(stream))
+
+
+def w4a16_moe_gather(X, src_row, Xg, T: int, rows: int, H: int, stream=None) -> int:
+    return load().w4a16_moe_gather(_addr(X), _addr(src_row), _addr(Xg), T, rows, H, _stream(stream))
+
+
+def w4a16_moe_combine(Y, weights, pos, out, T: int, top_k: int, H: int, stream=None) -> int:
+    return load().w4a16_moe_combine(_addr(Y), _addr(weights), _addr(pos), _addr(out), T, top_k, H,
+                                    _stream(stream))
+
+
+def w4a16_moe_workspace_size(T: int, E: int, top_k: int, H: int, I: int) -> int:
+    return int(load().w4a16_moe_workspace_size(T, E, top_k, H, I))
+
+
+def w4a16_moe_layer(X, logits, Wt_up: Sequence, S_up: Sequence, Wt_down: Sequence, S_down: Sequence, out,
+                    T: int, E: int, top_k: int, H: int, I: int, G: int, act: int, workspace, workspace_bytes: int,
+                    stream=None) -> int:
+    return load().w4a16_moe_layer(_addr(X), _addr(logits), _ptr_array(Wt_up), _ptr_array(S_up),
+                                  _ptr_array(Wt_down), _ptr_array(S_down), _addr(out), T, E, top_k, H, I, G, act,
+                                  _addr(workspace), workspace_bytes, _stream(stream))
+
+
+def w4a16_get_valid_tactics(M: int, N: int, K: int, G: int):
+    """(status, [tactic ids]) for a shape."""
+    count = ctypes.c_int32(0)
+    arr = (ctypes.c_int32 * 64)()
+    rc = load().w4a16_get_valid_tactics(M, N, K, G, arr, 64, ctypes.byref(count))
+    return rc, [arr[i] for i in range(min(count.value, 64))]
+
+
+def w4a16_tactic_launch_info(M: int, N: int, K: int, G: int, tactic: int):
+    info = LaunchInfo()
+    rc = load().w4a16_tactic_launch_info(M, N, K, G, tactic, ctypes.byref(info))
+    return rc, info
+
+
+def w4a16_set_tactic(M: int, N: int, K: int, G: int, tactic: int) -> int:
+    return load().w4a16_set_tactic(M, N, K, G, tactic)
+
+
+def w4a16_get_tactic(M: int, N: int, K: int, G: int) -> int:
+    t = ctypes.c_int32(-1)
+    rc = load().w4a16_get_tactic(M, N, K, G, ctypes.byref(t))
+    _check(rc, "w4a16_get_tactic")
+    return t.value
+
+
+def w4a16_clear_tactics() -> int:
+    return load().w4a16_clear_tactics()
+
+
+def w4a16_autotune(A, Wt, S, C, M: int, N: int, K: int, G: int, reps: int = 20, flush=None, flush_bytes: int = 0,
+                   stream=None):
+    """(status, best tactic id, its mean microseconds per launch)."""
+    best = ctypes.c_int32(0)
+    us = ctypes.c_float(0.0)
+    if flush is not None and not flush_bytes:
+        flush_bytes = flush.numel() * flush.element_size()
+    rc = load().w4a16_autotune(_addr(A), _addr(Wt), _addr(S), _addr(C), M, N, K, G, reps, _addr(flush), flush_bytes,
+                               ctypes.byref(best), ctypes.byref(us), _stream(stream))
+    return rc, best.value, us.value
+
+
+def w8a16_tiled_bytes(K: int, N: int) -> int:
+    return int(load().w8a16_tiled_bytes(K, N))
+
+
+def w8a16_repack(q, wt, K: int, N: int, stream=None) -> int:
+    return load().w8a16_repack(_addr(q), _addr(wt), K, N, _stream(stream))
+
+
+def w8a16_gemm(A, Wt8, S, C, M: int, N: int, K: int, G: int, stream=None) -> int:
+    return load().w8a16_gemm(_addr(A), _addr(Wt8), _addr(S), _addr(C), M, N, K, G, _stream(stream))
+
+
+def w8a16_gemm_launch_info(M: int, N: int, K: int, G: int):
+    info = LaunchInfo()
+    rc = load().w8a16_gemm_launch_info(M, N, K, G, ctypes.byref(info))
+    return rc, info
 
 
 def w4a16_gemm_launch_info(M: int, N: int, K: int, G: int):
@@ -271,6 +419,47 @@ def grouped_gemm(A, wts: Sequence, Ss: Sequence, offsets, N: int, G: int, out=No
     C = out if out is not None else torch.empty((rows, N), dtype=torch.float16, device=A.device)
     _check(w4a16_grouped_gemm(A.contiguous(), list(wts), [s.contiguous() for s in Ss], offsets, C, len(wts),
                               rows, N, K, G, stream), "w4a16_grouped_gemm")
+    return C
+
+
+def moe_layer(X, logits, wts_up: Sequence, Ss_up: Sequence, wts_down: Sequence, Ss_down: Sequence, top_k: int,
+              I: int, G: int, act: int, workspace=None, out=None, stream=None):
+    """The INT4 mixture-of-experts layer: out [T, H] from hidden states X [T, H] fp16 and router logits
+    [T, E] fp16 with per-expert tiled weights and scales (up: H -> I, down: I -> H). The workspace
+    (uint8, at least w4a16_moe_workspace_size bytes) is allocated here when not given."""
+    import torch
+    _require_cuda(X, logits)
+    T, H = X.shape
+    E = logits.shape[1]
+    need = w4a16_moe_workspace_size(T, E, top_k, H, I)
+    if need < 0:
+        raise W4A16Error(ERR_INVALID_ARG, "w4a16_moe_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=X.device)
+    C = out if out is not None else torch.empty((T, H), dtype=torch.float16, device=X.device)
+    _check(w4a16_moe_layer(X.contiguous(), logits.contiguous(), list(wts_up), [s.contiguous() for s in Ss_up],
+                           list(wts_down), [s.contiguous() for s in Ss_down], C, T, E, top_k, H, I, G, act,
+                           workspace, workspace.numel(), stream), "w4a16_moe_layer")
+    return C
+
+
+def repack_w8(q, stream=None):
+    """int8 codes [K, N] (device) -> the 8-bit tiled layout (flat uint8)."""
+    import torch
+    _require_cuda(q)
+    K, N = q.shape
+    wt = torch.empty(w8a16_tiled_bytes(K, N), dtype=torch.uint8, device=q.device)
+    _check(w8a16_repack(q.contiguous(), wt, K, N, stream), "w8a16_repack")
+    return wt
+
+
+def gemm_w8(A, wt8, S, N: int, G: int, out=None, stream=None):
+    """C [M, N] fp16 = A [M, K] fp16 x (8-bit codes in the tiled layout) * scales S."""
+    import torch
+    _require_cuda(A, wt8, S)
+    M, K = A.shape
+    C = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _check(w8a16_gemm(A.contiguous(), wt8, S.contiguous(), C, M, N, K, G, stream), "w8a16_gemm")
     return C
 
 

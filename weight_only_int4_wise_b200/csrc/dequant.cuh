@@ -1,4 +1,4 @@
-// int4 -> fp16 decoding of the tiled weight layout (include/w4a16.h): each
+// int4 (and 8-bit) -> fp16 decoding of the tiled weight layouts (include/w4a16.h): each
 // 32-bit word holds eight signed codes of one column, nibble i holding
 // k_local {0,2,4,6,1,3,5,7}[i], so that the decoder below yields (k, k+1)
 // pairs in natural order.
@@ -56,6 +56,21 @@ __device__ __forceinline__ uint4 decode_word(uint32_t x) {
     out.y = h2_bits(__hfma2(bits_h2(t0), sixteenth, bias_hi));
     out.z = h2_bits(__hsub2(bits_h2(b1), bias_lo));
     out.w = h2_bits(__hfma2(bits_h2(t1), sixteenth, bias_hi));
+    return out;
+}
+
+// Four signed 8-bit codes of one word (byte b = k_local b) -> two fp16 pairs
+// (q0, q1) * s and (q2, q3) * s. Flipping the sign bit of each byte gives
+// c + 128 in [0, 255]; placed under the exponent byte of 1024 (0x64) it reads as
+// the fp16 number 1024 + c + 128, exactly, and subtracting 1152 leaves c.
+__device__ __forceinline__ uint2 dequant_word8(uint32_t x, __half2 s2) {
+    const uint32_t u = x ^ 0x80808080u;
+    const uint32_t lo = __byte_perm(u, 0x64646464u, 0x4140u);  // bytes (u0, 0x64, u1, 0x64)
+    const uint32_t hi = __byte_perm(u, 0x64646464u, 0x4342u);  // bytes (u2, 0x64, u3, 0x64)
+    const __half2 bias = bits_h2(0x64806480u);                 // 1152, 1152
+    uint2 out;
+    out.x = h2_bits(__hmul2(__hsub2(bits_h2(lo), bias), s2));
+    out.y = h2_bits(__hmul2(__hsub2(bits_h2(hi), bias), s2));
     return out;
 }
 

@@ -44,6 +44,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <unordered_map>
 
 #include "../../include/w4a16.h"
 #include "dequant.cuh"
@@ -56,7 +57,7 @@ __device__ int g_status;  // latched device-side error (0 = none)
 
 constexpr int kTileN = 128;                 // weight columns per CTA (MMA M)
 constexpr int kTileK = 64;                  // K per pipeline stage
-constexpr int kRawBytes = 4096;             // int4 codes of one 128 x 64 tile
+constexpr int kRawBytes = 4096;             // int4 codes of one 128 x 64 tile (8-bit codes: twice that)
 constexpr int kSlotCols = kTileK / 2;       // TMEM columns of one dequantised 128 x 64 fp16 tile
 constexpr int kGroupWarps = 4;             // one dequantisation group: the 4 TMEM lane quadrants
 constexpr int kAhead = 2;                  // stages of its own a dequantising thread loads ahead
@@ -83,6 +84,7 @@ struct Params {
     int32_t vec_out;    // C rows start on 16-byte boundaries (16-byte output stores)
     long long wait_limit;   // bound of every device wait, in SM clock cycles
     int32_t stall_stage;    // test aid: the dequantising warps withhold this stage's ready signal (< 0: never)
+    int32_t act;            // W4A16_ACT_*: elementwise activation of the fp16 result (no K split)
 };
 
 // One ring of LS stages. Stage s owns, in shared memory, an activation tile
@@ -110,6 +112,29 @@ struct Layout {
 };
 
 __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
+
+// Epilogue value: the fp32 accumulator rounded to fp16 (the product's result),
+// then, for the expert layer's up projection, the activation evaluated in fp32
+// on that fp16 value and rounded to fp16 again. GELU in both of its usual
+// forms: x * Phi(x) with Phi the normal CDF (erf form), and the tanh
+// approximation with the cubic term 0.044715 x^3. Both are written without
+// the sum 1 + (something near -1) that loses all of fp32's digits for negative
+// x: Phi(x) = erfc(-x / sqrt 2) / 2, and (1 + tanh u) / 2 = 1 / (1 + e^(-2u)).
+__device__ __forceinline__ __half epilogue_value(float acc, int act) {
+    const __half h = __float2half_rn(acc);
+    if (act == W4A16_ACT_IDENTITY) return h;
+    const float x = __half2float(h);
+    float y;
+    if (act == W4A16_ACT_RELU) {
+        y = fmaxf(x, 0.f);
+    } else if (act == W4A16_ACT_GELU_ERF) {
+        y = 0.5f * x * erfcf(x * -0.70710678118654752f);
+    } else {
+        const float u = 0.79788456080286536f * (x + 0.044715f * x * x * x);
+        y = x / (1.f + expf(-2.f * u));
+    }
+    return __float2half_rn(y);
+}
 
 // Bounded wait on an mbarrier phase. Returns false if the CTA is aborting or
 // the wait ran out (which starts the abort). The bound is counted in SM clock
@@ -175,10 +200,16 @@ __device__ __forceinline__ bool warp_drain_phase(uint64_t* bar, uint32_t parity)
 }
 
 // OG: G is a multiple of 64, so a stage lies inside one scale group.
-template <int BN, int LS, int TMEM_COLS, int MINB, int DQ, bool OG>
+// BITS: 4 for the int4 tiled layout, 8 for the 8-bit code layout (W8A16): a
+// stage's tile is 4 or 8 KB, and a thread loads 2 or 4 16-byte chunks of its
+// column per stage; everything after the decode is the same.
+template <int BN, int LS, int TMEM_COLS, int MINB, int DQ, bool OG, int BITS>
 __global__ void __launch_bounds__(threads_for(DQ), MINB)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ Params p) {
     using L = Layout<BN, LS, TMEM_COLS>;
+    static_assert(BITS == 4 || BITS == 8, "int4 or 8-bit codes");
+    constexpr int kTileBytes = BITS == 4 ? kRawBytes : 2 * kRawBytes;  // one 128 x 64 tile of codes
+    constexpr int kChunks = BITS / 2;                                  // 16-byte chunks per column and stage
     constexpr int kScales = OG ? 1 : 8;  // scale registers per stage and thread
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base_addr = smem_addr(smem_raw);
@@ -267,16 +298,16 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
     // that reads a register whose load is in flight waits for that load.
     // kk is the first k of the next stage to load, gk = floor(kk / G).
     // (A padded column past N reads column 0's scales; its codes are 0.)
-    const uint8_t* wcol = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kRawBytes + j * 16;
+    const uint8_t* wcol = p.wt[expert] + static_cast<int64_t>(nt) * p.KT * kTileBytes + j * 16;
     const __half* scol = p.sc[expert] + (col_ok ? n : 0);
     int li = grp;
     int kk = (kb + grp) * kTileK;
     int gk = kk / p.G;
-    auto load_next = [&](uint4 (&r)[2], __half (&sv)[kScales]) {
+    auto load_next = [&](uint4 (&r)[kChunks], __half (&sv)[kScales]) {
         if (li < nst) {
-            const uint8_t* src = wcol + static_cast<int64_t>(kb + li) * kRawBytes;
-            r[0] = ld_nc_v4(src);
-            r[1] = ld_nc_v4(src + kRawBytes / 2);
+            const uint8_t* src = wcol + static_cast<int64_t>(kb + li) * kTileBytes;
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) r[c] = ld_nc_v4(src + c * 2048);
             if constexpr (OG) {
                 sv[0] = __ldg(scol + static_cast<int64_t>(min(gk, p.ngroups - 1)) * p.N);
             } else {
@@ -292,7 +323,8 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
                 }
             }
         } else {
-            r[0] = r[1] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) r[c] = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int q = 0; q < kScales; ++q) sv[q] = __float2half(0.f);
         }
@@ -300,7 +332,7 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         kk += kTileK * DQ;
         while ((gk + 1) * p.G <= kk) ++gk;
     };
-    uint4 rq0[2], rq1[2];
+    uint4 rq0[kChunks], rq1[kChunks];
     __half sq0[kScales], sq1[kScales];
     if (warp >= 2) {
         if (!p.prefetch) grid_dependency_wait();  // weights and scales may come from the previous kernel
@@ -340,11 +372,11 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
             // L2 kPrefetchStages ahead, so that the dequantising threads' own
             // loads (issued only kAhead of their stages ahead) find it there.
             // (The ring's first LS activation tiles go out before the prefetches.)
-            const uint8_t* wtile = p.wt[expert] + (static_cast<int64_t>(nt) * p.KT + kb) * kRawBytes;
+            const uint8_t* wtile = p.wt[expert] + (static_cast<int64_t>(nt) * p.KT + kb) * kTileBytes;
             const int first = min(nst, LS);
             for (int i = 0; i < first; ++i) issue_act(i);
             for (int i = 0; i < min(nst, kPrefetchStages + first); ++i)
-                bulk_prefetch_l2(wtile + static_cast<int64_t>(i) * kRawBytes, kRawBytes);
+                bulk_prefetch_l2(wtile + static_cast<int64_t>(i) * kTileBytes, kTileBytes);
             int issued = first;
             for (; issued < nst; ++issued) {
                 const int i = issued;
@@ -353,7 +385,7 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
                     break;
                 issue_act(i);
                 if (i + kPrefetchStages < nst)
-                    bulk_prefetch_l2(wtile + static_cast<int64_t>(i + kPrefetchStages) * kRawBytes, kRawBytes);
+                    bulk_prefetch_l2(wtile + static_cast<int64_t>(i + kPrefetchStages) * kTileBytes, kTileBytes);
             }
             // Every issued copy must land before the CTA's shared memory is released.
             for (int i = max(0, issued - LS); i < issued; ++i)
@@ -405,17 +437,31 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
         // One stage: decode the codes and scales held in (r, sv), refill them
         // with the thread's stage kAhead of its stages later, store the fp16
         // weights into the stage's TMEM slot and arrive. False when aborting.
-        auto stage = [&](int i, uint4 (&r)[2], __half (&sv)[kScales]) -> bool {
+        auto stage = [&](int i, uint4 (&r)[kChunks], __half (&sv)[kScales]) -> bool {
             const int s = i % LS;
-            const uint32_t raw[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
-            uint32_t v[2][16];  // k 0..31, k 32..63
+            uint32_t v[2][16];  // (k, k+1) pairs: k 0..31, k 32..63
+            if constexpr (BITS == 4) {
+                const uint32_t raw[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const uint4 o = dequant_word(raw[q], __half2half2(sv[OG ? 0 : q]));
-                v[q >> 2][4 * (q & 3)] = o.x;
-                v[q >> 2][4 * (q & 3) + 1] = o.y;
-                v[q >> 2][4 * (q & 3) + 2] = o.z;
-                v[q >> 2][4 * (q & 3) + 3] = o.w;
+                for (int q = 0; q < 8; ++q) {  // word q: k 8q .. 8q+7
+                    const uint4 o = dequant_word(raw[q], __half2half2(sv[OG ? 0 : q]));
+                    v[q >> 2][4 * (q & 3)] = o.x;
+                    v[q >> 2][4 * (q & 3) + 1] = o.y;
+                    v[q >> 2][4 * (q & 3) + 2] = o.z;
+                    v[q >> 2][4 * (q & 3) + 3] = o.w;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {  // chunk c: k 16c .. 16c+15
+                    const uint32_t raw[4] = {r[c].x, r[c].y, r[c].z, r[c].w};
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {  // word w: k 16c+4w .. +3, scale word (16c+4w)/8
+                        const uint2 o = dequant_word8(raw[w], __half2half2(sv[OG ? 0 : 2 * c + (w >> 1)]));
+                        const int pr = 8 * c + 2 * w;  // index of the pair (k, k+1) with k = 16c+4w
+                        v[pr >> 4][pr & 15] = o.x;
+                        v[pr >> 4][(pr & 15) + 1] = o.y;
+                    }
+                }
             }
             load_next(r, sv);
             // (Columns past N hold code 0 in the tiled layout and get scale 0: v is 0.)
@@ -470,12 +516,23 @@ __global__ void __launch_bounds__(threads_for(DQ), MINB)
                     tmem_ld_32x32b_x16(tmem_acc + tlane + c * 16, v);
                     if (two) tmem_ld_32x32b_x16(tmem_acc + tlane + (c + DQ) * 16, w);
                     tmem_ld_wait();
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) stile[(c * 16 + t) * kTileN + j] = __float2half_rn(__uint_as_float(v[t]));
-                    if (two) {
+                    const int act = p.act;
+                    if (act == W4A16_ACT_IDENTITY) {
 #pragma unroll
                         for (int t = 0; t < 16; ++t)
-                            stile[((c + DQ) * 16 + t) * kTileN + j] = __float2half_rn(__uint_as_float(w[t]));
+                            stile[(c * 16 + t) * kTileN + j] = __float2half_rn(__uint_as_float(v[t]));
+                        if (two) {
+#pragma unroll
+                            for (int t = 0; t < 16; ++t)
+                                stile[((c + DQ) * 16 + t) * kTileN + j] = __float2half_rn(__uint_as_float(w[t]));
+                        }
+                    } else {
+                        for (int t = 0; t < 16; ++t)
+                            stile[(c * 16 + t) * kTileN + j] = epilogue_value(__uint_as_float(v[t]), act);
+                        if (two) {
+                            for (int t = 0; t < 16; ++t)
+                                stile[((c + DQ) * 16 + t) * kTileN + j] = epilogue_value(__uint_as_float(w[t]), act);
+                        }
                     }
                 }
             }
@@ -580,11 +637,13 @@ struct Variant {
     int nominal_per_sm;  // the residency the variant is sized for (used when no device is present)
     int tmem_cols;       // TMEM columns each resident CTA allocates
     int smem;
-    const void* fn[2];  // [0]: G a multiple of 64 (one scale per stage), [1]: any G
-    int (*launch[2])(const CUtensorMap&, const Params&, dim3, int, int, cudaStream_t);
+    // [2 * (8-bit codes) + (any G)]: forms for int4 / 8-bit codes, with G a multiple
+    // of 64 (one scale per stage) or any G
+    const void* fn[4];
+    int (*launch[4])(const CUtensorMap&, const Params&, dim3, int, int, cudaStream_t);
 };
 
-template <int BN, int LS, int TC, int MINB, int DQ, bool OG>
+template <int BN, int LS, int TC, int MINB, int DQ, bool OG, int BITS>
 int launch_variant(const CUtensorMap& map, const Params& p, dim3 grid, int cluster_x, int smem, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -605,7 +664,7 @@ int launch_variant(const CUtensorMap& map, const Params& p, dim3 grid, int clust
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, w4a16_gemm_kernel<BN, LS, TC, MINB, DQ, OG>, map, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, w4a16_gemm_kernel<BN, LS, TC, MINB, DQ, OG, BITS>, map, p);
     return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
@@ -616,9 +675,12 @@ Variant make_variant() {
                    MINB,
                    TC,
                    Layout<BN, LS, TC>::kAlloc,
-                   {reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB, DQ, true>),
-                    reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB, DQ, false>)},
-                   {&launch_variant<BN, LS, TC, MINB, DQ, true>, &launch_variant<BN, LS, TC, MINB, DQ, false>}};
+                   {reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB, DQ, true, 4>),
+                    reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB, DQ, false, 4>),
+                    reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB, DQ, true, 8>),
+                    reinterpret_cast<const void*>(&w4a16_gemm_kernel<BN, LS, TC, MINB, DQ, false, 8>)},
+                   {&launch_variant<BN, LS, TC, MINB, DQ, true, 4>, &launch_variant<BN, LS, TC, MINB, DQ, false, 4>,
+                    &launch_variant<BN, LS, TC, MINB, DQ, true, 8>, &launch_variant<BN, LS, TC, MINB, DQ, false, 8>}};
 }
 
 // Token tiles and their pipeline depths: small tiles keep two CTAs per SM; the
@@ -642,7 +704,7 @@ const Variant& variant_for(int bn) {
 
 struct DeviceState {
     bool ready = false;
-    int ctas_per_sm[kNumVariants] = {};
+    int ctas_per_sm[2][kNumVariants] = {};  // [8-bit codes][variant]
 };
 
 int prepare_device(DeviceState** out) {
@@ -653,10 +715,12 @@ int prepare_device(DeviceState** out) {
     std::lock_guard<std::mutex> lock(mu);
     DeviceState& st = states[dev];
     if (!st.ready) {
-        for (int i = 0; i < kNumVariants; ++i) {
-            const Variant& v = kVariants[i];
+        for (int i = 0; i < 2 * kNumVariants; ++i) {
+            const Variant& v = kVariants[i % kNumVariants];
+            const int b8 = i / kNumVariants;
             int n = 1 << 30;
-            for (const void* fn : v.fn) {
+            for (int f = 2 * b8; f < 2 * b8 + 2; ++f) {
+                const void* fn = v.fn[f];
                 if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess ||
                     cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                          cudaSharedmemCarveoutMaxShared) != cudaSuccess)
@@ -678,7 +742,7 @@ int prepare_device(DeviceState** out) {
                 n = std::min(n, 512 / v.tmem_cols);  // every resident CTA holds its TMEM columns
             }
             if (n < 1) return W4A16_ERR_UNSUPPORTED;
-            st.ctas_per_sm[i] = n;
+            st.ctas_per_sm[b8][i % kNumVariants] = n;
         }
         st.ready = true;
     }
@@ -716,15 +780,20 @@ struct Plan {
     int ctas_per_sm;
 };
 
-int plan_dense(int64_t M, int64_t N, int64_t K, Plan* plan, bool need_device) {
-    const int bn = token_tile_for(M);
+// bn_force / splits_force > 0 select a tactic's token tile and K split (the
+// split only with a single token tile, a power of two that leaves every
+// cluster rank at least two K stages); 0 takes the heuristic.
+int plan_dense(int64_t M, int64_t N, int64_t K, Plan* plan, bool need_device, int bn_force = 0,
+               int splits_force = 0, int bits = 4) {
+    const int bn = bn_force > 0 ? bn_force : token_tile_for(M);
+    if (variant_for(bn).bn != bn) return W4A16_ERR_UNSUPPORTED;
     const int vi = variant_index(bn);
     int per_sm = kVariants[vi].nominal_per_sm, sms = 148;
     if (need_device) {
         DeviceState* st = nullptr;
         int rc = prepare_device(&st);
         if (rc) return rc;
-        per_sm = st->ctas_per_sm[vi];
+        per_sm = st->ctas_per_sm[bits == 8 ? 1 : 0][vi];
         sms = sm_count();
     }
     const int64_t NT = (N + kTileN - 1) / kTileN;
@@ -732,7 +801,12 @@ int plan_dense(int64_t M, int64_t N, int64_t K, Plan* plan, bool need_device) {
     const int64_t KT = (K + kTileK - 1) / kTileK;
     if (NT > 65535 || MT > 65535) return W4A16_ERR_UNSUPPORTED;
     int splits = 1;
-    if (MT == 1) {
+    if (splits_force > 0) {
+        if ((splits_force & (splits_force - 1)) || splits_force > 8 ||
+            (splits_force > 1 && (MT != 1 || KT < 2 * splits_force)))
+            return W4A16_ERR_UNSUPPORTED;
+        splits = splits_force;
+    } else if (MT == 1) {
         const int64_t slots = static_cast<int64_t>(sms) * per_sm;
         while (splits < 8 && NT * splits * 2 <= slots && KT >= splits * 4) splits *= 2;
     }
@@ -756,7 +830,7 @@ int plan_grouped(int64_t E, int64_t total_rows, int64_t N, int64_t K, Plan* plan
         DeviceState* st = nullptr;
         int rc = prepare_device(&st);
         if (rc) return rc;
-        per_sm = st->ctas_per_sm[vi];
+        per_sm = st->ctas_per_sm[0][vi];
     }
     const int64_t NT = (N + kTileN - 1) / kTileN;
     const int64_t slots = total_rows / bn + E;  // >= sum over experts of ceil(rows_e / bn)
@@ -783,7 +857,134 @@ void fill_info(const Plan& plan, w4a16_launch_info* info) {
     info->ctas_per_sm = plan.ctas_per_sm;
 }
 
+// ---------------------------------------------------------------- tactics
+// A tactic is one launch form of w4a16_gemm for a shape (the plugin page's
+// getValidTactics / setTactic): the skinny kernel with a given K split, K
+// halves and ring depth (M <= 16 only), or the tensor-core kernel with a given
+// token tile and K split. Ids are 1-based positions in the shape's list of
+// valid forms, skinny forms first; 0 means the built-in heuristic.
+struct Choice {
+    bool skinny;
+    SkinnyPlan sk;
+    Plan tc;
+};
+
+constexpr int kTileChoices[] = {16, 32, 64, 128, 192, 256};
+
+void enumerate_tactics(int64_t M, int64_t N, int64_t K, int64_t G, bool need_device, Choice* out, int* count,
+                       int capacity) {
+    int n = 0;
+    auto push = [&](const Choice& c) {
+        if (n < capacity) out[n] = c;
+        ++n;
+    };
+    if (M <= kSkinnyMaxM) {
+        for (int kh = 1; kh <= 2; ++kh)
+            for (int splits = 1; splits <= 8; ++splits)
+                for (int deep = 0; deep <= 1; ++deep) {
+                    Choice c{};
+                    c.skinny = true;
+                    if (skinny_plan_fill(M, N, K, G, splits, kh, deep, &c.sk) == W4A16_OK) push(c);
+                }
+    }
+    for (int bn : kTileChoices)
+        for (int splits = 1; splits <= 8; splits *= 2) {
+            Choice c{};
+            c.skinny = false;
+            if (plan_dense(M, N, K, &c.tc, need_device, bn, splits) == W4A16_OK) push(c);
+        }
+    *count = n;
+}
+
+constexpr int kMaxTactics = 64;
+
+int tactic_choice(int64_t M, int64_t N, int64_t K, int64_t G, int tactic, bool need_device, Choice* out) {
+    Choice all[kMaxTactics];
+    int n = 0;
+    enumerate_tactics(M, N, K, G, need_device, all, &n, kMaxTactics);
+    if (tactic < 1 || tactic > n || tactic > kMaxTactics) return W4A16_ERR_INVALID_ARG;
+    *out = all[tactic - 1];
+    return W4A16_OK;
+}
+
+struct TacticKey {
+    int dev;
+    int64_t M, N, K, G;
+    bool operator==(const TacticKey& o) const {
+        return dev == o.dev && M == o.M && N == o.N && K == o.K && G == o.G;
+    }
+};
+struct TacticKeyHash {
+    size_t operator()(const TacticKey& k) const {
+        uint64_t h = static_cast<uint64_t>(k.dev) * 0x9E3779B97F4A7C15ull;
+        for (int64_t v : {k.M, k.N, k.K, k.G}) h = (h ^ static_cast<uint64_t>(v)) * 0x100000001B3ull;
+        return static_cast<size_t>(h);
+    }
+};
+struct TacticEntry {
+    int tactic;
+    Choice choice;
+};
+
+std::mutex g_tactic_mu;
+std::unordered_map<TacticKey, TacticEntry, TacticKeyHash> g_tactics;
+std::atomic<int> g_tactic_count{0};  // lets the GEMM skip the lookup while the table is empty
+
+int current_device() {
+    int dev = 0;
+    return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
+// The table's choice for a shape on the current device, if it holds one.
+bool lookup_tactic(int64_t M, int64_t N, int64_t K, int64_t G, Choice* out, int* tactic) {
+    if (g_tactic_count.load(std::memory_order_acquire) == 0) return false;
+    const TacticKey key{current_device(), M, N, K, G};
+    std::lock_guard<std::mutex> lock(g_tactic_mu);
+    auto it = g_tactics.find(key);
+    if (it == g_tactics.end()) return false;
+    *out = it->second.choice;
+    if (tactic) *tactic = it->second.tactic;
+    return true;
+}
+
+void store_tactic(int64_t M, int64_t N, int64_t K, int64_t G, int tactic, const Choice& c) {
+    const TacticKey key{current_device(), M, N, K, G};
+    std::lock_guard<std::mutex> lock(g_tactic_mu);
+    if (tactic == 0) {
+        g_tactics.erase(key);
+    } else {
+        g_tactics[key] = TacticEntry{tactic, c};
+    }
+    g_tactic_count.store(static_cast<int>(g_tactics.size()), std::memory_order_release);
+}
+
+// The table's tactic for the shape, else the heuristic: the skinny kernel for
+// decode-sized M, the tensor-core kernel otherwise.
+int choose(int64_t M, int64_t N, int64_t K, int64_t G, bool need_device, Choice* c) {
+    if (lookup_tactic(M, N, K, G, c, nullptr)) return W4A16_OK;
+    c->skinny = skinny_plan(M, N, K, G, &c->sk) == W4A16_OK;
+    if (c->skinny) return W4A16_OK;
+    return plan_dense(M, N, K, &c->tc, need_device);
+}
+
+void fill_info_skinny(const SkinnyPlan& sk, w4a16_launch_info* info) {
+    info->token_tile = 8 * sk.mt;
+    info->k_splits = sk.splits;
+    info->grid_x = sk.grid_x;
+    info->grid_y = sk.grid_y;
+    info->grid_z = 1;
+    info->threads_per_cta = sk.threads;
+    info->smem_bytes = sk.smem;
+    info->ctas_per_sm = (228 * 1024) / (sk.smem + 1024) < 2 ? (228 * 1024) / (sk.smem + 1024) : 2;
+}
+
 }  // namespace
+
+int launch_choice(const Choice& c, const w4a16_half* A_dev, const uint8_t* Wt_dev, const w4a16_half* S_dev,
+                  w4a16_half* C_dev, int64_t M, int64_t N, int64_t K, int64_t G, cudaStream_t stream);
+int dense_launch(const Plan& plan, int bits, const w4a16_half* A_dev, const uint8_t* Wt_dev,
+                 const w4a16_half* S_dev, w4a16_half* C_dev, int64_t M, int64_t N, int64_t K, int64_t G,
+                 cudaStream_t stream);
 
 int activation_map(CUtensorMap* map, const void* A, int64_t rows, int64_t K, int box_rows) {
     // A small per-thread cache: the encoder costs more than the rest of a
@@ -896,6 +1097,7 @@ extern "C" const char* w4a16_status_string(int status) {
         case W4A16_ERR_CUDA: return "CUDA runtime error";
         case W4A16_ERR_TIMEOUT: return "bounded device wait ran out";
         case W4A16_ERR_BAD_OFFSETS: return "malformed expert offsets";
+        case W4A16_ERR_BAD_ROUTING: return "expert id or gathered-row index out of range";
         default: return "unknown status";
     }
 }
@@ -911,22 +1113,13 @@ extern "C" int w4a16_gemm_launch_info(int64_t M, int64_t N, int64_t K, int64_t G
     if (rc) return rc;
     if (M >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
     const bool dev = check_device() == W4A16_OK;
-    SkinnyPlan sk;
-    if (skinny_plan(M, N, K, G, &sk) == W4A16_OK) {
-        info->token_tile = 8 * sk.mt;
-        info->k_splits = sk.splits;
-        info->grid_x = sk.grid_x;
-        info->grid_y = sk.grid_y;
-        info->grid_z = 1;
-        info->threads_per_cta = sk.threads;
-        info->smem_bytes = sk.smem;
-        info->ctas_per_sm = (228 * 1024) / (sk.smem + 1024) < 2 ? (228 * 1024) / (sk.smem + 1024) : 2;
-        return W4A16_OK;
-    }
-    Plan plan;
-    rc = plan_dense(M, N, K, &plan, dev);
+    Choice c;
+    rc = choose(M, N, K, G, dev, &c);
     if (rc) return rc;
-    fill_info(plan, info);
+    if (c.skinny)
+        fill_info_skinny(c.sk, info);
+    else
+        fill_info(c.tc, info);
     return W4A16_OK;
 }
 
@@ -956,13 +1149,25 @@ extern "C" int w4a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt_dev, const 
     if (M == 0) return W4A16_OK;
     rc = check_device();
     if (rc) return rc;
-    SkinnyPlan sk;
-    if (skinny_plan(M, N, K, G, &sk) == W4A16_OK)
-        return skinny_launch(sk, A_dev, Wt_dev, S_dev, C_dev, M, N, K, G, static_cast<cudaStream_t>(stream));
-    Plan plan;
-    rc = plan_dense(M, N, K, &plan, true);
+    Choice c;
+    rc = choose(M, N, K, G, true, &c);
     if (rc) return rc;
+    return launch_choice(c, A_dev, Wt_dev, S_dev, C_dev, M, N, K, G, static_cast<cudaStream_t>(stream));
+}
 
+namespace w4a16 {
+
+int launch_choice(const Choice& c, const w4a16_half* A_dev, const uint8_t* Wt_dev, const w4a16_half* S_dev,
+                  w4a16_half* C_dev, int64_t M, int64_t N, int64_t K, int64_t G, cudaStream_t stream) {
+    if (c.skinny) return skinny_launch(c.sk, A_dev, Wt_dev, S_dev, C_dev, M, N, K, G, stream);
+    return dense_launch(c.tc, 4, A_dev, Wt_dev, S_dev, C_dev, M, N, K, G, stream);
+}
+
+// The tensor-core kernel on a dense product, int4 (bits = 4) or 8-bit codes.
+int dense_launch(const Plan& plan, int bits, const w4a16_half* A_dev, const uint8_t* Wt_dev,
+                 const w4a16_half* S_dev, w4a16_half* C_dev, int64_t M, int64_t N, int64_t K, int64_t G,
+                 cudaStream_t stream) {
+    int rc;
     Params p;
     std::memset(&p, 0, sizeof(p));
     p.wt[0] = Wt_dev;
@@ -987,14 +1192,19 @@ extern "C" int w4a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt_dev, const 
     rc = activation_map(&map, A_dev, M, K, plan.bn);
     if (rc) return rc;
     const Variant& v = variant_for(plan.bn);
-    return v.launch[(G % kTileK) ? 1 : 0](map, p, plan.grid, plan.splits, v.smem, static_cast<cudaStream_t>(stream));
+    return v.launch[(bits == 8 ? 2 : 0) + ((G % kTileK) ? 1 : 0)](map, p, plan.grid, plan.splits, v.smem, stream);
 }
 
-extern "C" int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const* Wt, const w4a16_half* const* S,
-                                  const int32_t* offsets_dev, w4a16_half* C_dev, int64_t E, int64_t total_rows,
-                                  int64_t N, int64_t K, int64_t G, void* stream) {
+}  // namespace w4a16
+
+namespace w4a16 {
+
+int grouped_gemm_act(const w4a16_half* A_dev, const uint8_t* const* Wt, const w4a16_half* const* S,
+                     const int32_t* offsets_dev, w4a16_half* C_dev, int64_t E, int64_t total_rows, int64_t N,
+                     int64_t K, int64_t G, int act, cudaStream_t stream) {
     if (!A_dev || !Wt || !S || !offsets_dev || !C_dev || E <= 0 || E > W4A16_MAX_EXPERTS || total_rows < 0)
         return W4A16_ERR_INVALID_ARG;
+    if (act < W4A16_ACT_IDENTITY || act > W4A16_ACT_GELU_TANH) return W4A16_ERR_INVALID_ARG;
     int rc = check_shape(N, K, G);
     if (rc) return rc;
     if (total_rows >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
@@ -1033,12 +1243,30 @@ extern "C" int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const*
     p.prefetch = 0;  // expert weights are read only after the offsets, which follow the wait
     p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
     p.stall_stage = g_stall_stage.load(std::memory_order_relaxed);
+    p.act = act;
 
     CUtensorMap map;
     rc = activation_map(&map, A_dev, total_rows, K, plan.bn);
     if (rc) return rc;
     const Variant& v = variant_for(plan.bn);
-    return v.launch[(G % kTileK) ? 1 : 0](map, p, plan.grid, 1, v.smem, static_cast<cudaStream_t>(stream));
+    return v.launch[(G % kTileK) ? 1 : 0](map, p, plan.grid, 1, v.smem, stream);  // int4 forms
+}
+
+}  // namespace w4a16
+
+extern "C" int w4a16_grouped_gemm(const w4a16_half* A_dev, const uint8_t* const* Wt, const w4a16_half* const* S,
+                                  const int32_t* offsets_dev, w4a16_half* C_dev, int64_t E, int64_t total_rows,
+                                  int64_t N, int64_t K, int64_t G, void* stream) {
+    return grouped_gemm_act(A_dev, Wt, S, offsets_dev, C_dev, E, total_rows, N, K, G, W4A16_ACT_IDENTITY,
+                            static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int w4a16_grouped_gemm_act(const w4a16_half* A_dev, const uint8_t* const* Wt,
+                                      const w4a16_half* const* S, const int32_t* offsets_dev, w4a16_half* C_dev,
+                                      int64_t E, int64_t total_rows, int64_t N, int64_t K, int64_t G, int act,
+                                      void* stream) {
+    return grouped_gemm_act(A_dev, Wt, S, offsets_dev, C_dev, E, total_rows, N, K, G, act,
+                            static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int w4a16_device_status(int clear) {
@@ -1052,12 +1280,176 @@ extern "C" int w4a16_device_status(int clear) {
     }
     const int vs = skinny_device_status(clear != 0);
     const int vq = quant_device_status(clear != 0);
-    if (vs < 0 || vq < 0) return W4A16_ERR_CUDA;
-    return v != 0 ? v : (vs != 0 ? vs : vq);
+    const int vm = moe_device_status(clear != 0);
+    if (vs < 0 || vq < 0 || vm < 0) return W4A16_ERR_CUDA;
+    return v != 0 ? v : (vs != 0 ? vs : (vq != 0 ? vq : vm));
 }
 
 extern "C" int w4a16_set_fault_injection(int64_t stall_stage, int64_t wait_limit_cycles) {
     g_stall_stage.store(stall_stage < 0 || stall_stage > (1 << 30) ? -1 : static_cast<int>(stall_stage));
     g_wait_limit.store(wait_limit_cycles > 0 ? static_cast<long long>(wait_limit_cycles) : kTimeoutCycles);
     return W4A16_OK;
+}
+
+// ---------------------------------------------------------------- tactics
+extern "C" int w4a16_get_valid_tactics(int64_t M, int64_t N, int64_t K, int64_t G, int32_t* tactics,
+                                       int32_t capacity, int32_t* count) {
+    if (!count || M <= 0 || capacity < 0 || (capacity > 0 && !tactics)) return W4A16_ERR_INVALID_ARG;
+    int rc = check_shape(N, K, G);
+    if (rc) return rc;
+    if (M >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    Choice all[kMaxTactics];
+    int n = 0;
+    enumerate_tactics(M, N, K, G, check_device() == W4A16_OK, all, &n, kMaxTactics);
+    n = std::min(n, kMaxTactics);
+    for (int i = 0; i < n && i < capacity; ++i) tactics[i] = i + 1;
+    *count = n;
+    return W4A16_OK;
+}
+
+extern "C" int w4a16_tactic_launch_info(int64_t M, int64_t N, int64_t K, int64_t G, int32_t tactic,
+                                        w4a16_launch_info* info) {
+    if (!info || M <= 0) return W4A16_ERR_INVALID_ARG;
+    int rc = check_shape(N, K, G);
+    if (rc) return rc;
+    if (M >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    Choice c;
+    rc = tactic_choice(M, N, K, G, tactic, check_device() == W4A16_OK, &c);
+    if (rc) return rc;
+    if (c.skinny)
+        fill_info_skinny(c.sk, info);
+    else
+        fill_info(c.tc, info);
+    return W4A16_OK;
+}
+
+extern "C" int w4a16_set_tactic(int64_t M, int64_t N, int64_t K, int64_t G, int32_t tactic) {
+    if (M <= 0 || tactic < 0) return W4A16_ERR_INVALID_ARG;
+    int rc = check_shape(N, K, G);
+    if (rc) return rc;
+    if (M >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    Choice c{};
+    if (tactic > 0) {
+        rc = tactic_choice(M, N, K, G, tactic, check_device() == W4A16_OK, &c);
+        if (rc) return rc;
+    }
+    store_tactic(M, N, K, G, tactic, c);
+    return W4A16_OK;
+}
+
+extern "C" int w4a16_get_tactic(int64_t M, int64_t N, int64_t K, int64_t G, int32_t* tactic) {
+    if (!tactic) return W4A16_ERR_INVALID_ARG;
+    Choice c;
+    int t = 0;
+    *tactic = lookup_tactic(M, N, K, G, &c, &t) ? t : 0;
+    return W4A16_OK;
+}
+
+extern "C" int w4a16_clear_tactics(void) {
+    std::lock_guard<std::mutex> lock(g_tactic_mu);
+    g_tactics.clear();
+    g_tactic_count.store(0, std::memory_order_release);
+    return W4A16_OK;
+}
+
+extern "C" int w4a16_autotune(const w4a16_half* A_dev, const uint8_t* Wt_dev, const w4a16_half* S_dev,
+                              w4a16_half* C_dev, int64_t M, int64_t N, int64_t K, int64_t G, int32_t reps,
+                              void* flush_dev, int64_t flush_bytes, int32_t* best_tactic, float* best_us,
+                              void* stream) {
+    if (!A_dev || !Wt_dev || !S_dev || !C_dev || !best_tactic || M <= 0 || reps < 1 || reps > 10000 ||
+        flush_bytes < 0 || (flush_bytes > 0 && !flush_dev))
+        return W4A16_ERR_INVALID_ARG;
+    int rc = check_shape(N, K, G);
+    if (rc) return rc;
+    if (M >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    if (!aligned16(A_dev) || !aligned16(Wt_dev) || !aligned16(S_dev) ||
+        (reinterpret_cast<uintptr_t>(C_dev) & 1u))
+        return W4A16_ERR_MISALIGNED;
+    rc = check_device();
+    if (rc) return rc;
+    Choice all[kMaxTactics];
+    int n = 0;
+    enumerate_tactics(M, N, K, G, true, all, &n, kMaxTactics);
+    n = std::min(n, kMaxTactics);
+    if (n == 0) return W4A16_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaEvent_t e0 = nullptr, e1 = nullptr;
+    if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) {
+        if (e0) cudaEventDestroy(e0);
+        return W4A16_ERR_CUDA;
+    }
+    float best = 0.f;
+    int best_id = 0;
+    rc = W4A16_OK;
+    for (int i = 0; i < n && rc == W4A16_OK; ++i) {
+        // one untimed launch (first-use setup), then the timed ones
+        rc = launch_choice(all[i], A_dev, Wt_dev, S_dev, C_dev, M, N, K, G, st);
+        float total_ms = 0.f;
+        if (rc == W4A16_OK && flush_bytes > 0) {
+            // each timed launch starts with the weights out of L2
+            for (int r = 0; r < reps && rc == W4A16_OK; ++r) {
+                float ms = 0.f;
+                if (cudaMemsetAsync(flush_dev, r & 0xFF, static_cast<size_t>(flush_bytes), st) != cudaSuccess ||
+                    cudaEventRecord(e0, st) != cudaSuccess) {
+                    rc = W4A16_ERR_CUDA;
+                    break;
+                }
+                rc = launch_choice(all[i], A_dev, Wt_dev, S_dev, C_dev, M, N, K, G, st);
+                if (rc == W4A16_OK && (cudaEventRecord(e1, st) != cudaSuccess || cudaEventSynchronize(e1) != cudaSuccess ||
+                                       cudaEventElapsedTime(&ms, e0, e1) != cudaSuccess))
+                    rc = W4A16_ERR_CUDA;
+                total_ms += ms;
+            }
+        } else if (rc == W4A16_OK) {
+            if (cudaEventRecord(e0, st) != cudaSuccess) rc = W4A16_ERR_CUDA;
+            for (int r = 0; r < reps && rc == W4A16_OK; ++r)
+                rc = launch_choice(all[i], A_dev, Wt_dev, S_dev, C_dev, M, N, K, G, st);
+            if (rc == W4A16_OK && (cudaEventRecord(e1, st) != cudaSuccess || cudaEventSynchronize(e1) != cudaSuccess ||
+                                   cudaEventElapsedTime(&total_ms, e0, e1) != cudaSuccess))
+                rc = W4A16_ERR_CUDA;
+        }
+        const float us = total_ms * 1000.f / static_cast<float>(reps);
+        if (rc == W4A16_OK && (best_id == 0 || us < best)) {
+            best = us;
+            best_id = i + 1;
+        }
+    }
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    if (rc) return rc;
+    store_tactic(M, N, K, G, best_id, all[best_id - 1]);
+    *best_tactic = best_id;
+    if (best_us) *best_us = best;
+    return W4A16_OK;
+}
+
+// ---------------------------------------------------------------- W8A16
+extern "C" int w8a16_gemm_launch_info(int64_t M, int64_t N, int64_t K, int64_t G, w4a16_launch_info* info) {
+    if (!info || M <= 0) return W4A16_ERR_INVALID_ARG;
+    int rc = check_shape(N, K, G);
+    if (rc) return rc;
+    if (M >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    Plan plan;
+    rc = plan_dense(M, N, K, &plan, check_device() == W4A16_OK, 0, 0, 8);
+    if (rc) return rc;
+    fill_info(plan, info);
+    return W4A16_OK;
+}
+
+extern "C" int w8a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt8_dev, const w4a16_half* S_dev,
+                          w4a16_half* C_dev, int64_t M, int64_t N, int64_t K, int64_t G, void* stream) {
+    if (!A_dev || !Wt8_dev || !S_dev || !C_dev || M < 0) return W4A16_ERR_INVALID_ARG;
+    int rc = check_shape(N, K, G);
+    if (rc) return rc;
+    if (M >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    if (!aligned16(A_dev) || !aligned16(Wt8_dev) || !aligned16(S_dev) ||
+        (reinterpret_cast<uintptr_t>(C_dev) & 1u))
+        return W4A16_ERR_MISALIGNED;
+    if (M == 0) return W4A16_OK;
+    rc = check_device();
+    if (rc) return rc;
+    Plan plan;
+    rc = plan_dense(M, N, K, &plan, true, 0, 0, 8);
+    if (rc) return rc;
+    return dense_launch(plan, 8, A_dev, Wt8_dev, S_dev, C_dev, M, N, K, G, static_cast<cudaStream_t>(stream));
 }

@@ -33,6 +33,14 @@ int make_half_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_
 // buffers skip the encoder.
 int activation_map(CUtensorMap* map, const void* A, int64_t rows, int64_t K, int box_rows);
 
+// The grouped-expert GEMM with an activation epilogue (w4a16_grouped_gemm_act).
+int grouped_gemm_act(const w4a16_half* A_dev, const uint8_t* const* Wt, const w4a16_half* const* S,
+                     const int32_t* offsets_dev, w4a16_half* C_dev, int64_t E, int64_t total_rows, int64_t N,
+                     int64_t K, int64_t G, int act, cudaStream_t stream);
+
+// The expert-layer kernels' latched device status (0 = none, -1 if it could not be read).
+int moe_device_status(bool clear);
+
 // The quantiser kernel's latched device status (0 = none, -1 if it could not be read).
 int quant_device_status(bool clear);
 
@@ -54,6 +62,12 @@ struct SkinnyPlan {
 
 // W4A16_OK and a plan, or W4A16_ERR_UNSUPPORTED if the shape needs the general kernel.
 int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan);
+
+// The skinny plan for a given K split (1..8 CTAs per cluster), K halves per CTA
+// (1 or 2; 2 only for one token tile) and ring depth (deep = 0: four blocks in
+// flight per CTA, 1: eight). W4A16_ERR_UNSUPPORTED when that form does not
+// exist for the shape (more splits than 128-deep K blocks, shared memory).
+int skinny_plan_fill(int64_t M, int64_t N, int64_t K, int64_t G, int splits, int kh, int deep, SkinnyPlan* plan);
 
 // The skinny kernel's latched device status (0 = none, -1 if it could not be read).
 int skinny_device_status(bool clear);

@@ -70,6 +70,31 @@ __global__ void repack_kernel(const uint8_t* __restrict__ wp, uint32_t* __restri
     }
 }
 
+// One thread per 16-byte chunk of the 8-bit tiled layout: chunk (tile, h, j)
+// holds the codes k_local = 16h .. 16h+15 of column j, byte b = k_local 16h + b.
+__global__ void repack8_kernel(const int8_t* __restrict__ q, uint4* __restrict__ wt, int64_t K, int64_t N,
+                               int64_t KT, int64_t total_chunks) {
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total_chunks;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t tile = idx >> 9;        // 512 chunks per 8192-byte tile
+        const int32_t r = static_cast<int32_t>(idx & 511);
+        const int32_t h = r >> 7;             // 128 chunks per 16-row quarter
+        const int32_t j = r & 127;            // column inside the tile
+        const int64_t nt = tile / KT, kt = tile - nt * KT;
+        const int64_t n = nt * 128 + j;
+        const int64_t kbase = kt * 64 + 16 * h;
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        if (n < N) {
+#pragma unroll
+            for (int b = 0; b < 16; ++b) {
+                const int64_t k = kbase + b;
+                if (k < K) w[b >> 2] |= static_cast<uint32_t>(static_cast<uint8_t>(q[k * N + n])) << (8 * (b & 3));
+            }
+        }
+        wt[idx] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 static int grid_for(int64_t work) {
     int64_t blocks = (work + 255) / 256;
     if (blocks > 148 * 32) blocks = 148 * 32;
@@ -112,5 +137,22 @@ extern "C" int w4a16_repack(const uint8_t* wp_dev, uint8_t* wt_dev, int64_t K, i
     const int64_t words = w4a16_tiled_bytes(K, N) / 4;
     repack_kernel<<<grid_for(words), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         wp_dev, reinterpret_cast<uint32_t*>(wt_dev), K, N, KT, words);
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+extern "C" int64_t w8a16_tiled_bytes(int64_t K, int64_t N) {
+    if (K <= 0 || N <= 0) return 0;
+    return ((N + 127) / 128) * ((K + 63) / 64) * 8192;
+}
+
+extern "C" int w8a16_repack(const int8_t* q_dev, uint8_t* wt_dev, int64_t K, int64_t N, void* stream) {
+    if (!q_dev || !wt_dev || K <= 0 || N <= 0) return W4A16_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(wt_dev) & 15) return W4A16_ERR_MISALIGNED;
+    int rc = check_device();
+    if (rc) return rc;
+    const int64_t KT = (K + 63) / 64;
+    const int64_t chunks = w8a16_tiled_bytes(K, N) / 16;
+    repack8_kernel<<<grid_for(chunks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        q_dev, reinterpret_cast<uint4*>(wt_dev), K, N, KT, chunks);
     return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }

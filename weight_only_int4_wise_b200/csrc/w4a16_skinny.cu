@@ -325,6 +325,49 @@ int smem_bytes(int kh, int depth, int mt, int splits, int act_stride, int scale_
 
 }  // namespace
 
+int skinny_plan_fill(int64_t M, int64_t N, int64_t K, int64_t G, int splits, int kh, int deep, SkinnyPlan* plan) {
+    if (M < 1 || M > kSkinnyMaxM) return W4A16_ERR_UNSUPPORTED;
+    const int64_t NT = (N + 127) / 128;
+    const int64_t KT = (K + 63) / 64;
+    const int64_t KB = (KT + 1) / 2;
+    const int mt = M <= 8 ? 1 : 2;
+    if (NT > 65535 || splits < 1 || splits > 8 || splits > KB) return W4A16_ERR_UNSUPPORTED;
+    if (kh < 1 || kh > 2 || (kh == 2 && mt != 1)) return W4A16_ERR_UNSUPPORTED;  // compiled forms only
+    const int64_t nbmax = (KB + splits - 1) / splits;
+    const int dmax = 8 / kh;  // 128-deep blocks in flight per thread: 8 per CTA
+    const int depth = deep ? dmax : dmax / 2;
+    const int64_t krange = nbmax * kBlockK;
+    const int64_t stride = krange + 8;
+    const int64_t rows = krange / G + 2;
+    const int64_t bytes =
+        smem_bytes(kh, depth, mt, splits, static_cast<int>(stride), static_cast<int>(rows));
+    if (bytes > 200 * 1024) return W4A16_ERR_UNSUPPORTED;
+    // floor(k / G) as a multiply-shift over the padded K range. With
+    // magic = (2^32 + e) / G, 0 <= e < G, k * magic / 2^32 = k / G + k * e / (G * 2^32),
+    // which floors to floor(k / G) whenever k * e < 2^32 (the fractional part of
+    // k / G is at most (G - 1) / G). Otherwise every k is checked.
+    const uint64_t magic = ((uint64_t(1) << 32) + static_cast<uint64_t>(G) - 1) / static_cast<uint64_t>(G);
+    if (magic > 0xFFFFFFFFull) return W4A16_ERR_UNSUPPORTED;
+    const uint64_t e = magic * static_cast<uint64_t>(G) - (uint64_t(1) << 32);
+    const uint64_t kend = static_cast<uint64_t>(KB * kBlockK);
+    if (e != 0 && kend > ((uint64_t(1) << 32) - 1) / e) {
+        for (int64_t k = 0; k < KB * kBlockK; k += 8)
+            if (static_cast<int64_t>((static_cast<uint64_t>(k) * magic) >> 32) != k / G) return W4A16_ERR_UNSUPPORTED;
+    }
+    plan->splits = splits;
+    plan->depth = depth;
+    plan->act_stride = static_cast<int>(stride);
+    plan->scale_rows = static_cast<int>(rows < (K + G - 1) / G ? rows : (K + G - 1) / G);
+    plan->smem = smem_bytes(kh, depth, mt, plan->splits, plan->act_stride, plan->scale_rows);
+    plan->mt = mt;
+    plan->threads = kh * kSkThreads;
+    plan->grid_x = splits;
+    plan->grid_y = static_cast<int>(NT);
+    plan->g_magic = static_cast<uint32_t>(magic);
+    plan->post_scale = (G % kBlockK) == 0 ? 1 : 0;
+    return W4A16_OK;
+}
+
 int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan) {
     if (M < 1 || M > kSkinnyMaxM) return W4A16_ERR_UNSUPPORTED;
     const int64_t NT = (N + 127) / 128;
@@ -345,48 +388,15 @@ int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan) {
     if (splits < 1) splits = 1;
     for (;;) {
         const int64_t nbmax = (KB + splits - 1) / splits;
-        // Blocks in flight per thread: 8 per CTA (4 per K half with two halves),
-        // all of them for short K ranges.
+        // All eight blocks in flight per CTA for long K ranges, half of them
+        // for short ones.
         const int kh = k_halves(mt, nbmax);
         const int64_t nbh = (nbmax + kh - 1) / kh;  // blocks of one K half
-        const int dmax = 8 / kh;
-        const int depth = nbh <= dmax / 2 ? dmax / 2 : dmax;
-        const int64_t krange = nbmax * kBlockK;
-        const int64_t stride = krange + 8;
-        const int64_t rows = krange / G + 2;
-        const int64_t bytes = smem_bytes(kh, depth, mt, static_cast<int>(splits), static_cast<int>(stride),
-                                         static_cast<int>(rows));
-        if (bytes <= 200 * 1024) {
-            plan->splits = static_cast<int>(splits);
-            plan->depth = depth;
-            plan->act_stride = static_cast<int>(stride);
-            plan->scale_rows = static_cast<int>(rows < (K + G - 1) / G ? rows : (K + G - 1) / G);
-            plan->smem = smem_bytes(kh, depth, mt, plan->splits, plan->act_stride, plan->scale_rows);
-            plan->mt = mt;
-            plan->threads = kh * kSkThreads;
-            plan->grid_x = static_cast<int>(splits);
-            plan->grid_y = static_cast<int>(NT);
-            break;
-        }
+        const int deep = nbh <= (8 / kh) / 2 ? 0 : 1;
+        if (skinny_plan_fill(M, N, K, G, static_cast<int>(splits), kh, deep, plan) == W4A16_OK) return W4A16_OK;
         if (splits >= 8 || splits >= KB) return W4A16_ERR_UNSUPPORTED;
         ++splits;
     }
-    if (NT > 65535) return W4A16_ERR_UNSUPPORTED;
-    // floor(k / G) as a multiply-shift over the padded K range. With
-    // magic = (2^32 + e) / G, 0 <= e < G, k * magic / 2^32 = k / G + k * e / (G * 2^32),
-    // which floors to floor(k / G) whenever k * e < 2^32 (the fractional part of
-    // k / G is at most (G - 1) / G). Otherwise every k is checked.
-    const uint64_t magic = ((uint64_t(1) << 32) + static_cast<uint64_t>(G) - 1) / static_cast<uint64_t>(G);
-    if (magic > 0xFFFFFFFFull) return W4A16_ERR_UNSUPPORTED;
-    const uint64_t e = magic * static_cast<uint64_t>(G) - (uint64_t(1) << 32);
-    const uint64_t kend = static_cast<uint64_t>(KB * kBlockK);
-    if (e != 0 && kend > ((uint64_t(1) << 32) - 1) / e) {
-        for (int64_t k = 0; k < KB * kBlockK; k += 8)
-            if (static_cast<int64_t>((static_cast<uint64_t>(k) * magic) >> 32) != k / G) return W4A16_ERR_UNSUPPORTED;
-    }
-    plan->g_magic = static_cast<uint32_t>(magic);
-    plan->post_scale = (G % kBlockK) == 0 ? 1 : 0;
-    return W4A16_OK;
 }
 
 int skinny_device_status(bool clear) {

@@ -162,6 +162,9 @@ CONFIGS: Dict[str, dict] = {
     # the whole mixture-of-experts layer around the grouped product (up 4096 -> 14336,
     # down 14336 -> 4096), routed by its own logits
     "moe_layer":   dict(kind="moe", E=8, top_k=2, tokens=512, H=4096, I=14336, G=128, seed=6),
+    # the 8-bit code variant (W8A16) at the decode and prefill sizes
+    "w8_decode_m16": dict(kind="dense8", M=16, K=4096, N=4096, G=128, seed=7),
+    "w8_prefill":    dict(kind="dense8", M=2048, K=4096, N=4096, G=128, seed=8),
 }
 
 
@@ -172,4 +175,6 @@ def make(name: str):
         return dense(name=name, **cfg)
     if kind == "moe":
         return moe(name=name, **cfg)
+    if kind == "dense8":
+        return dense8(name=name, **cfg)
     return grouped(name=name, **cfg)
