@@ -64,8 +64,10 @@ enum {
     W4A16_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
     W4A16_ERR_TIMEOUT = 5,      /* device status: a bounded wait inside a kernel ran out */
     W4A16_ERR_BAD_OFFSETS = 6,  /* device status: expert offsets not 0 = o[0] <= ... <= o[E] = rows */
-    W4A16_ERR_BAD_ROUTING = 7   /* device status: an expert id out of range or repeated within a token,
+    W4A16_ERR_BAD_ROUTING = 7,  /* device status: an expert id out of range or repeated within a token,
                                    or a gathered-row index out of range */
+    W4A16_ERR_SCRATCH_TOO_SMALL = 8  /* w4a16_moe_layer_static: the shape needs more intermediates than
+                                        the library's static scratch holds */
 };
 
 /* Elementwise activations of the expert layer (Int4 Moe Plugin page,
@@ -236,6 +238,42 @@ int w4a16_moe_layer(const w4a16_half* X_dev, const w4a16_half* logits_dev, const
                     const w4a16_half* const* S_up, const uint8_t* const* Wt_down, const w4a16_half* const* S_down,
                     w4a16_half* out_dev, int64_t T, int64_t E, int64_t top_k, int64_t H, int64_t I, int64_t G,
                     int act, void* workspace_dev, int64_t workspace_bytes, void* stream);
+
+/* The whole layer without a caller workspace: the same six steps as
+ * w4a16_moe_layer (same kernels, bit-identical results), with the
+ * intermediates in a fixed region of device memory that the library itself
+ * owns, w4a16_moe_static_scratch_bytes() = 8 MiB per device, created with the
+ * library's device code when the CUDA runtime loads it. The plugin pages have
+ * no counterpart of this entry point.
+ *
+ * For callers that cannot provide or obtain device memory at call time: an
+ * engine whose execute step was promised a zero-byte workspace when it was
+ * built, or C code that owns no device allocator. Allocating inside the call
+ * is no option for them (cudaMalloc synchronizes the device and may fail under
+ * memory pressure in the middle of a step); nothing here calls cudaMalloc,
+ * cudaFree or any other allocating routine.
+ *
+ * - The first call on a device looks up the region's device address
+ *   (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ *   first call on each device before any stream capture begins.
+ * - Shapes whose intermediates (w4a16_moe_workspace_size) exceed the region
+ *   are refused with W4A16_ERR_SCRATCH_TOO_SMALL before anything is enqueued;
+ *   at H = 4096 and I = 14336 the region holds about 180 gathered rows
+ *   (T * topK), a decode batch.
+ * - Nothing in the region needs to start at zero or survive between calls:
+ *   every intermediate is written before it is read within a call.
+ * - All calls on a device share the one region: two calls whose kernels may
+ *   overlap on the GPU (different streams, or different host threads, without
+ *   ordering between them) race on it and may return wrong results. Calls
+ *   ordered on one stream are safe.
+ * Arguments, other errors and T == 0 as for w4a16_moe_layer. */
+int w4a16_moe_layer_static(const w4a16_half* X_dev, const w4a16_half* logits_dev, const uint8_t* const* Wt_up,
+                           const w4a16_half* const* S_up, const uint8_t* const* Wt_down,
+                           const w4a16_half* const* S_down, w4a16_half* out_dev, int64_t T, int64_t E,
+                           int64_t top_k, int64_t H, int64_t I, int64_t G, int act, void* stream);
+
+/* Size in bytes of the static scratch region of w4a16_moe_layer_static. */
+int64_t w4a16_moe_static_scratch_bytes(void);
 
 /* Declares (enable != 0) or withdraws (enable == 0) the promise that no
  * kernel on the calling streams writes the tiled weights or the scales passed

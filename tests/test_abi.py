@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(8):
+    for code in range(9):
         assert w.status_string(code) != "unknown status"
     assert w.status_string(99) == "unknown status"
 
@@ -265,3 +265,14 @@ def test_w8_tiled_bytes_and_host_checks(lib):
     assert w.w8a16_repack(None, FAKE, 4, 4, stream=0) == w.ERR_INVALID_ARG
     rc, info = w.w8a16_gemm_launch_info(16, 4096, 4096, 128)
     assert rc == w.OK and info.token_tile == 16 and info.threads_per_cta == 320  # the tensor-core kernel
+
+
+def test_static_scratch_layer_host_checks(lib):
+    # the no-allocation expert layer refuses shapes beyond its static scratch before touching CUDA
+    assert w.w4a16_moe_static_scratch_bytes() == 8 << 20
+    ptrs = [FAKE] * 8
+    call = lambda T, H, I: w.w4a16_moe_layer_static(FAKE, FAKE, ptrs, ptrs, ptrs, ptrs, FAKE, T, 8, 2, H, I, 128,
+                                                     w.ACT_RELU, stream=0)
+    assert call(512, 4096, 14336) == w.ERR_SCRATCH_TOO_SMALL
+    assert call(4, 4096, 0) == w.ERR_INVALID_ARG
+    assert call(0, 4096, 14336) == w.OK

@@ -11,9 +11,9 @@ from ._lib import (  # noqa: F401
     w4a16_moe_workspace_size, w4a16_pack, w4a16_quantize, w4a16_repack, w4a16_set_fault_injection,
     w4a16_set_static_weights, w4a16_tiled_bytes, w4a16_unpack, w4a16_get_valid_tactics, w4a16_tactic_launch_info,
     w4a16_set_tactic, w4a16_get_tactic, w4a16_clear_tactics, w4a16_autotune, w8a16_tiled_bytes, w8a16_repack,
-    w8a16_gemm, w8a16_gemm_launch_info, repack_w8, gemm_w8,
+    w8a16_gemm, w8a16_gemm_launch_info, repack_w8, gemm_w8, w4a16_moe_layer_static, w4a16_moe_static_scratch_bytes,
 )
 from ._lib import (  # noqa: F401
     ACT_GELU_ERF, ACT_GELU_TANH, ACT_IDENTITY, ACT_RELU, ERR_BAD_OFFSETS, ERR_BAD_ROUTING, ERR_CUDA,
-    ERR_INVALID_ARG, ERR_MISALIGNED, ERR_TIMEOUT, ERR_UNSUPPORTED, OK,
+    ERR_INVALID_ARG, ERR_MISALIGNED, ERR_SCRATCH_TOO_SMALL, ERR_TIMEOUT, ERR_UNSUPPORTED, OK,
 )

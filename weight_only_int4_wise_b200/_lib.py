@@ -24,6 +24,7 @@ ERR_CUDA = 4
 ERR_TIMEOUT = 5
 ERR_BAD_OFFSETS = 6
 ERR_BAD_ROUTING = 7
+ERR_SCRATCH_TOO_SMALL = 8
 MAX_EXPERTS = 64
 MAX_TOPK = 8
 ACT_IDENTITY = 0
@@ -39,6 +40,7 @@ EXPORTED = [
     "w4a16_moe_workspace_size", "w4a16_moe_layer", "w4a16_get_valid_tactics", "w4a16_tactic_launch_info",
     "w4a16_set_tactic", "w4a16_get_tactic", "w4a16_clear_tactics", "w4a16_autotune",
     "w8a16_tiled_bytes", "w8a16_repack", "w8a16_gemm", "w8a16_gemm_launch_info",
+    "w4a16_moe_layer_static", "w4a16_moe_static_scratch_bytes",
 ]
 
 
@@ -112,6 +114,12 @@ def load() -> ctypes.CDLL:
                                         ctypes.POINTER(_vp), _vp, _i64, _i64, _i64, _i64, _i64, _i64, ctypes.c_int,
                                         _vp, _i64, _vp]
         lib.w4a16_moe_layer.restype = ctypes.c_int
+        lib.w4a16_moe_layer_static.argtypes = [_vp, _vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                                               ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _i64, _i64, _i64,
+                                               _i64, _i64, _i64, ctypes.c_int, _vp]
+        lib.w4a16_moe_layer_static.restype = ctypes.c_int
+        lib.w4a16_moe_static_scratch_bytes.argtypes = []
+        lib.w4a16_moe_static_scratch_bytes.restype = _i64
         lib.w8a16_tiled_bytes.argtypes = [_i64, _i64]
         lib.w8a16_tiled_bytes.restype = _i64
         lib.w8a16_repack.argtypes = [_vp, _vp, _i64, _i64, _vp]
@@ -306,6 +314,20 @@ def w8a16_gemm_launch_info(M: int, N: int, K: int, G: int):
     info = LaunchInfo()
     rc = load().w8a16_gemm_launch_info(M, N, K, G, ctypes.byref(info))
     return rc, info
+
+
+def w4a16_moe_layer_static(X, logits, Wt_up: Sequence, S_up: Sequence, Wt_down: Sequence, S_down: Sequence, out,
+                           T: int, E: int, top_k: int, H: int, I: int, G: int, act: int, stream=None) -> int:
+    """The expert layer without a workspace argument: its intermediates live in the library's
+    static per-device scratch (see include/w4a16.h for the limits and the race between
+    overlapping calls)."""
+    return load().w4a16_moe_layer_static(_addr(X), _addr(logits), _ptr_array(Wt_up), _ptr_array(S_up),
+                                         _ptr_array(Wt_down), _ptr_array(S_down), _addr(out), T, E, top_k, H, I,
+                                         G, act, _stream(stream))
+
+
+def w4a16_moe_static_scratch_bytes() -> int:
+    return int(load().w4a16_moe_static_scratch_bytes())
 
 
 def w4a16_gemm_launch_info(M: int, N: int, K: int, G: int):

@@ -1098,6 +1098,7 @@ extern "C" const char* w4a16_status_string(int status) {
         case W4A16_ERR_TIMEOUT: return "bounded device wait ran out";
         case W4A16_ERR_BAD_OFFSETS: return "malformed expert offsets";
         case W4A16_ERR_BAD_ROUTING: return "expert id or gathered-row index out of range";
+        case W4A16_ERR_SCRATCH_TOO_SMALL: return "shape needs more than the static scratch of the no-allocation entry point";
         default: return "unknown status";
     }
 }

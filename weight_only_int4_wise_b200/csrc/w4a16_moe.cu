@@ -22,6 +22,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/w4a16.h"
 #include "ptx.cuh"
@@ -488,4 +489,58 @@ extern "C" int w4a16_moe_layer(const w4a16_half* X_dev, const w4a16_half* logits
                                reinterpret_cast<w4a16_half*>(w.y), E, rows, H, I, G, W4A16_ACT_IDENTITY, s)))
         return rc;
     return moe_combine(reinterpret_cast<const w4a16_half*>(w.y), w.weights, w.pos, out_dev, T, top_k, H, s);
+}
+
+// ------------------------------------------------- no-allocation entry point
+// Some callers cannot hand the layer a workspace: an engine whose execute step
+// was promised a zero-byte workspace at build time, or C code that owns no
+// device memory pool. A cudaMalloc inside the call is no way out for them:
+// it synchronizes the device and can fail under memory pressure in the middle
+// of a step. w4a16_moe_layer_static therefore runs the same six steps in a
+// fixed region of device memory that belongs to this library (one per device,
+// created with the module), sized for decode-scale batches.
+namespace w4a16 {
+namespace {
+
+constexpr int64_t kStaticScratchBytes = int64_t(8) << 20;  // 8 MiB per device
+static __device__ __align__(256) uint8_t g_moe_scratch[kStaticScratchBytes];
+
+// Device address of g_moe_scratch, looked up once per device with that device
+// current; nullptr if the lookup failed.
+void* static_scratch() {
+    static std::mutex mu;
+    static void* ptr[64] = {};
+    static bool done[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_moe_scratch) != cudaSuccess) return nullptr;
+        ptr[dev] = p;
+        done[dev] = true;
+    }
+    return ptr[dev];
+}
+
+}  // namespace
+}  // namespace w4a16
+
+extern "C" int64_t w4a16_moe_static_scratch_bytes(void) { return w4a16::kStaticScratchBytes; }
+
+extern "C" int w4a16_moe_layer_static(const w4a16_half* X_dev, const w4a16_half* logits_dev,
+                                      const uint8_t* const* Wt_up, const w4a16_half* const* S_up,
+                                      const uint8_t* const* Wt_down, const w4a16_half* const* S_down,
+                                      w4a16_half* out_dev, int64_t T, int64_t E, int64_t top_k, int64_t H,
+                                      int64_t I, int64_t G, int act, void* stream) {
+    const int64_t need = w4a16_moe_workspace_size(T, E, top_k, H, I);
+    if (need < 0) return W4A16_ERR_INVALID_ARG;
+    if (need > w4a16::kStaticScratchBytes) return W4A16_ERR_SCRATCH_TOO_SMALL;
+    if (T == 0) return w4a16_moe_layer(X_dev, logits_dev, Wt_up, S_up, Wt_down, S_down, out_dev, T, E, top_k, H,
+                                       I, G, act, reinterpret_cast<void*>(uintptr_t(256)), need, stream);
+    if (check_device() != W4A16_OK) return W4A16_ERR_UNSUPPORTED;
+    void* scratch = w4a16::static_scratch();
+    if (!scratch) return W4A16_ERR_CUDA;
+    return w4a16_moe_layer(X_dev, logits_dev, Wt_up, S_up, Wt_down, S_down, out_dev, T, E, top_k, H, I, G, act,
+                           scratch, w4a16::kStaticScratchBytes, stream);
 }
