@@ -319,6 +319,36 @@ def run_ours(args):
     launch(1, 0)
     launch(16, 1)
     torch.cuda.synchronize()
+    # Launch forms. By default the library's built-in heuristic, whose choices for
+    # these two shapes were made for this alternating M=1 / M=16 sequence. With
+    # --tune-headline the autotuner picks each shape's fastest form on its own
+    # (back to back over the rotating copies); on B200 its M=16 choice (a deeper
+    # ring, 92 KB of shared memory) is faster alone but no longer shares an SM
+    # with the M=1 launch, and the alternating step got slower (17.8 against
+    # 15.5 us), so it stays opt-in.
+    w4.w4a16_clear_tactics()
+    tuned = {}
+    pinned = dict(tuple(int(x) for x in kv.split("=")) for kv in args.pin_tactics.split(",") if kv)
+    for m in M_STEP:
+        heur = w4.w4a16_gemm_launch_info(m, N_DIM, K_DIM, G_DIM)[1].as_dict()
+        if not args.tune_headline and m not in pinned:
+            tuned[f"M={m}"] = {"tactic": 0, "form": heur, "note": "built-in heuristic"}
+            continue
+        if m in pinned:
+            rc = w4.w4a16_set_tactic(m, N_DIM, K_DIM, G_DIM, pinned[m])
+            if rc:
+                raise RuntimeError(f"tactic {pinned[m]}: {w4.status_string(rc)}")
+            tuned[f"M={m}"] = {"tactic": pinned[m], "pinned": True, "heuristic_form": heur,
+                               "form": w4.w4a16_gemm_launch_info(m, N_DIM, K_DIM, G_DIM)[1].as_dict()}
+            continue
+        rc, best, best_us = w4.w4a16_autotune(As[0], wts, Ss, outs[m], m, N_DIM, K_DIM, G_DIM, reps=20)
+        if rc:
+            raise RuntimeError(f"autotune: {w4.status_string(rc)}")
+        tuned[f"M={m}"] = {"tactic": best, "tuner_us": round(best_us, 3), "heuristic_form": heur,
+                           "form": w4.w4a16_gemm_launch_info(m, N_DIM, K_DIM, G_DIM)[1].as_dict()}
+    launch(1, 0)
+    launch(16, 1)
+    torch.cuda.synchronize()
 
     def capture(nsteps, start):
         g = torch.cuda.CUDAGraph()
@@ -384,33 +414,66 @@ def run_ours(args):
     C1_d, C16_d = C_d[:1], C_d[1:]
     K_e2e = min(K, 2000)
 
-    # The step as a decode loop runs it: the host->device copy of the step's
-    # activations, the two GEMMs through the C entry point, the device->host copy
-    # of their results, recorded once into a CUDA graph of E2E_GRAPH_STEPS steps
-    # (rotating weight copies as in the timed region) and replayed; every step
-    # still moves its inputs in and its outputs out.
+    # The steps as a server runs independent batches: each step copies its
+    # activations in from pinned host memory, runs the two GEMMs through the C
+    # entry point and copies both results out to pinned host memory. The copies
+    # run on two more streams (one per direction, so the two copy engines work at
+    # once) into double buffers, so that step i's GEMMs overlap the copy-in of
+    # step i+1 and the copy-out of step i-1. E2E_GRAPH_STEPS steps
+    # (rotating weight copies as in the timed region) are recorded once into a
+    # CUDA graph and replayed; every step still moves its inputs in and its
+    # outputs out.
     E2E_GRAPH_STEPS = 16
     cgemm = w4.load().w4a16_gemm
-    a1, a16, c1, c16 = A1_d.data_ptr(), A16_d.data_ptr(), C1_d.data_ptr(), C16_d.data_ptr()
+    A_db = [A_d, torch.empty_like(A_d)]
+    C_db = [C_d, torch.empty_like(C_d)]
+    a_ptr = [(x[:1].data_ptr(), x[1:].data_ptr()) for x in A_db]
+    c_ptr = [(x[:1].data_ptr(), x[1:].data_ptr()) for x in C_db]
     wptr = [x.data_ptr() for x in wts]
     sptr = [x.data_ptr() for x in Ss]
+    in_stream, out_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)  # one copy engine per direction
 
-    def e2e_step(i):
-        st = torch.cuda.current_stream(dev).cuda_stream
-        r1, r2 = (2 * i) % R, (2 * i + 1) % R
-        A_d.copy_(A_h, non_blocking=True)
-        if cgemm(a1, wptr[r1], sptr[r1], c1, 1, N_DIM, K_DIM, G_DIM, st) or \
-                cgemm(a16, wptr[r2], sptr[r2], c16, 16, N_DIM, K_DIM, G_DIM, st):
-            raise RuntimeError("a GEMM call failed in the end-to-end loop")
-        C_h.copy_(C_d, non_blocking=True)
+    def e2e_steps(n):
+        comp = torch.cuda.current_stream(dev)
+        st = comp.cuda_stream
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+        ev_back = [torch.cuda.Event() for _ in range(n)]
+        in_stream.wait_stream(comp)
+        out_stream.wait_stream(comp)
 
-    for i in range(E2E_GRAPH_STEPS):
-        e2e_step(i)
+        def copy_in(i):
+            with torch.cuda.stream(in_stream):
+                if i >= 2:
+                    in_stream.wait_event(ev_out[i - 2])  # step i-2's GEMMs have read this buffer
+                A_db[i % 2].copy_(A_h, non_blocking=True)
+                ev_in[i].record(in_stream)
+
+        copy_in(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                copy_in(i + 1)
+            comp.wait_event(ev_in[i])
+            if i >= 2:
+                comp.wait_event(ev_back[i - 2])  # step i-2's results have left this buffer
+            r1, r2 = (2 * i) % R, (2 * i + 1) % R
+            if cgemm(a_ptr[b][0], wptr[r1], sptr[r1], c_ptr[b][0], 1, N_DIM, K_DIM, G_DIM, st) or \
+                    cgemm(a_ptr[b][1], wptr[r2], sptr[r2], c_ptr[b][1], 16, N_DIM, K_DIM, G_DIM, st):
+                raise RuntimeError("a GEMM call failed in the end-to-end loop")
+            ev_out[i].record(comp)
+            with torch.cuda.stream(out_stream):
+                out_stream.wait_event(ev_out[i])
+                C_h.copy_(C_db[b], non_blocking=True)
+                ev_back[i].record(out_stream)
+        comp.wait_stream(in_stream)
+        comp.wait_stream(out_stream)
+
+    e2e_steps(E2E_GRAPH_STEPS)
     torch.cuda.synchronize()
     g_e2e = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_e2e):
-        for i in range(E2E_GRAPH_STEPS):
-            e2e_step(i)
+        e2e_steps(E2E_GRAPH_STEPS)
     reps_e2e = max(1, K_e2e // E2E_GRAPH_STEPS)
     K_e2e = reps_e2e * E2E_GRAPH_STEPS
     for _ in range(3):
@@ -428,9 +491,12 @@ def run_ours(args):
     e2e = {"value": job_throughput(K_e2e * step_bytes(), world, e2e_sec) / 1e9, "unit": "GB/s",
            "h2d_bytes_per_step": sum(m * K_DIM * 2 for m in M_STEP),
            "d2h_bytes_per_step": sum(m * N_DIM * 2 for m in M_STEP), "steps": K_e2e,
-           "launch": f"CUDA graph of {E2E_GRAPH_STEPS} steps (copy in, two w4a16_gemm calls, copy out), replayed"}
+           "launch": f"CUDA graph of {E2E_GRAPH_STEPS} steps, replayed: per step one copy in (pinned host -> device), "
+                     "two w4a16_gemm calls, one copy out (device -> pinned host); copies on one stream per "
+                     "direction with double buffers overlap the neighbouring steps' GEMMs"}
 
-    extra = per_config(w4, dev) if (rank == 0 and not args.no_configs) else None
+    extra = per_config(w4, dev, tune=not args.no_tune) if (rank == 0 and not args.no_configs) else None
+    tactics = tactic_report(w4, dev) if (rank == 0 and not args.no_configs) else None
     peaks = load_peaks()
     achieved = K * step_bytes() / sec / 1e9  # per GPU: every launch in the step is the same kernel
     line = {
@@ -441,7 +507,10 @@ def run_ours(args):
                    "l2": f"inputs larger than L2: {R} rotating copies of weights+scales+activations "
                          f"({R * copy_bytes / 2 ** 20:.0f} MiB vs {l2 / 2 ** 20:.0f} MiB L2)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "static_weights": True, "launch": "CUDA graphs, programmatic dependent launch"},
+                   "static_weights": True,
+                   "launch": "CUDA graphs, programmatic dependent launch" +
+                             ("; launch forms from the library's autotuner at setup" if args.tune_headline
+                              else "; built-in launch heuristic")},
         "tflops": round(tflops, 3),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic_from_profile(),
@@ -451,13 +520,16 @@ def run_ours(args):
         "step_us": dict(step_stats, note="device time per step (one M=1 and one M=16 launch), 100 CUDA-graph "
                                          "replays of 20 steps, after the timed region"),
         "gpu_launches": world * 2 * K,
-        "launch": {f"M={m}": w4.w4a16_gemm_launch_info(m, N_DIM, K_DIM, G_DIM)[1].as_dict() for m in M_STEP},
+        "launch": {k: v["form"] for k, v in tuned.items()},
+        "tactics_at_setup": tuned,
         "clocks": clocks,
     }
     if rank == 0:
         line["cpu_baseline"] = None if args.no_cpu_baseline else cpu_baseline()
         if extra is not None:
             line["per_config"] = extra
+        if tactics is not None:
+            line["tactics"] = tactics
         print(json.dumps(line), flush=True)
     del g_main, g_rem
     if world > 1:
@@ -465,8 +537,71 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def per_config(w4, dev):
-    """Device time per launch for every workload family (context for the headline line)."""
+TACTIC_SHAPES = [(1, 4096, 4096), (16, 4096, 4096), (8, 4096, 14336), (8, 14336, 4096)]  # (M, K, N), G = 128
+
+
+def tactic_report(w4, dev):
+    """The tactic table on the decode launches and the MLP shapes: the autotuner
+    times every valid form the way the headline runs (back-to-back launches in a
+    CUDA graph over rotating weight copies larger than L2), then the heuristic's
+    form and the tuned one are timed again by the same replay as per_config.
+    The headline uses the heuristic; the table is emptied again afterwards."""
+    import torch
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20)
+    out = {}
+    for (M, K, N) in TACTIC_SHAPES:
+        G = G_DIM
+        c = workloads.dense(M, K, N, G, seed=1)
+        _, wt = w4.prepare_weights(torch.from_numpy(c.q).to(dev))
+        S = torch.from_numpy(c.S).to(dev)
+        A = torch.from_numpy(c.A).to(dev)
+        C = torch.empty((M, N), dtype=torch.float16, device=dev)
+        per = wt.numel() + S.numel() * 2
+        R = max(2, math.ceil(2 * l2 / per) + 1)
+        wts = [wt] + [wt.clone() for _ in range(R - 1)]
+        Ss = [S] + [S.clone() for _ in range(R - 1)]
+        w4.w4a16_clear_tactics()
+        heur = w4.w4a16_gemm_launch_info(M, N, K, G)[1].as_dict()
+        _, ids = w4.w4a16_get_valid_tactics(M, N, K, G)
+        forms = {t: w4.w4a16_tactic_launch_info(M, N, K, G, t)[1].as_dict() for t in ids}
+        heur_id = next((t for t in ids if forms[t] == heur), 0)
+        rc, best, best_us, times = w4.w4a16_autotune(A, wts, Ss, C, M, N, K, G, reps=20, with_times=True)
+        if rc:
+            raise RuntimeError(f"autotune: {w4.status_string(rc)}")
+
+        def graph_us():
+            def launch(r):
+                rc_ = w4.w4a16_gemm(A, wts[r], Ss[r], C, M, N, K, G)
+                if rc_:
+                    raise RuntimeError(w4.status_string(rc_))
+            launch(0)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(20):
+                    launch(i % R)
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            st = replay_stats(g, 20, 50)
+            del g
+            return st["median"]
+
+        tuned_graph = graph_us()  # the tuned entry is in the table now
+        w4.w4a16_clear_tactics()
+        heur_graph = graph_us()
+        out[f"M={M},K={K},N={N}"] = {
+            "tactics": len(ids), "heuristic": heur_id, "heuristic_form": heur,
+            "heuristic_tuner_us": round(times[heur_id - 1], 3) if heur_id else None,
+            "tuned": best, "tuned_form": forms[best], "tuned_tuner_us": round(best_us, 3),
+            "heuristic_graph_us": heur_graph, "tuned_graph_us": tuned_graph,
+            "tuner_us_by_tactic": [round(x, 2) for x in times]}
+    w4.w4a16_clear_tactics()
+    return out
+
+
+def per_config(w4, dev, tune=True):
+    """Device time per launch for every workload family (context for the headline line).
+    Dense W4A16 shapes run the autotuned launch form (unless tune is False)."""
     import torch
     peaks = load_peaks()
     l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20)
@@ -475,6 +610,7 @@ def per_config(w4, dev):
         if name == "tiny":
             continue
         c = workloads.make(name)
+        tactic = None
         if cfg["kind"] == "dense":
             _, wt = w4.prepare_weights(torch.from_numpy(c.q).to(dev))
             S = torch.from_numpy(c.S).to(dev)
@@ -490,6 +626,12 @@ def per_config(w4, dev):
                 rc = w4.w4a16_gemm(A_, wt_, S_, C_, M, N, K, G)
                 if rc:
                     raise RuntimeError(w4.status_string(rc))
+            tactic = 0
+            if tune:  # the library's autotuner over the same rotating copies, as a user tunes at setup
+                rc, tactic, _ = w4.w4a16_autotune(A, [b[0] for b in bufs], [b[1] for b in bufs], C, M, N, K, G,
+                                                  reps=20)
+                if rc:
+                    raise RuntimeError(f"autotune: {w4.status_string(rc)}")
             fl = flops(M, N, K)
             by = algorithmic_bytes(M, N, K, G)
         elif cfg["kind"] == "dense8":
@@ -576,6 +718,8 @@ def per_config(w4, dev):
                      "bound": "hbm" if by / (peaks["hbm_gbs"] * 1e9) >= fl / (peaks["bf16_tflops"] * 1e12)
                      else "tensor", "rotating_copies": R, "timing": f"median of {st['reps']} CUDA-graph replays of "
                                                                   f"{n} launches each"}
+        if tactic is not None:
+            out[name]["tactic"] = tactic
         del g
     out["quantize"] = quantize_timing(w4, dev, peaks, l2)
     status = w4.device_status(clear=True)
@@ -679,7 +823,26 @@ def run_profile(args):
         print(f"profiled quantize: {args.launches} launches")
         return
     c = workloads.make(args.profile)
-    if isinstance(c, workloads.DenseCase):
+    kind = workloads.CONFIGS[args.profile]["kind"]
+    if kind == "dense8":
+        wt = w4.repack_w8(torch.from_numpy(c.q).to(dev))
+        A, S = torch.from_numpy(c.A).to(dev), torch.from_numpy(c.S).to(dev)
+        C = torch.empty((c.M, c.N), dtype=torch.float16, device=dev)
+        for _ in range(args.launches):
+            w4.gemm_w8(A, wt, S, c.N, c.G, out=C)
+    elif kind == "moe":
+        up = [w4.prepare_weights(torch.from_numpy(c.q_up[e]).to(dev))[1] for e in range(c.E)]
+        down = [w4.prepare_weights(torch.from_numpy(c.q_down[e]).to(dev))[1] for e in range(c.E)]
+        su = [torch.from_numpy(x).to(dev) for x in c.S_up]
+        sd = [torch.from_numpy(x).to(dev) for x in c.S_down]
+        X, lg = torch.from_numpy(c.X).to(dev), torch.from_numpy(c.logits).to(dev)
+        for _ in range(args.launches):
+            w4.moe_layer(X, lg, up, su, down, sd, c.top_k, c.I, c.G, w4.ACT_GELU_ERF)
+    elif isinstance(c, workloads.DenseCase):
+        if args.tactic:
+            rc = w4.w4a16_set_tactic(c.M, c.N, c.K, c.G, args.tactic)
+            if rc:
+                raise RuntimeError(f"tactic {args.tactic}: {w4.status_string(rc)}")
         _, wt = w4.prepare_weights(torch.from_numpy(c.q).to(dev))
         A, S = torch.from_numpy(c.A).to(dev), torch.from_numpy(c.S).to(dev)
         C = torch.empty((c.M, c.N), dtype=torch.float16, device=dev)
@@ -707,9 +870,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config timings")
+    ap.add_argument("--no-tune", action="store_true",
+                    help="per-config timings with the built-in heuristic instead of autotuned launch forms")
+    ap.add_argument("--tune-headline", action="store_true",
+                    help="autotune the two headline shapes at setup (each on its own) instead of the heuristic")
     ap.add_argument("--profile", choices=sorted(workloads.CONFIGS) + ["quantize"],
                     help="only launch this workload (for ncu)")
     ap.add_argument("--launches", type=int, default=4, help="launches in --profile mode")
+    ap.add_argument("--tactic", type=int, default=0, help="--profile mode: pin this tactic id for the shape")
+    ap.add_argument("--pin-tactics", default="",
+                    help="headline mode: 'M=id,...' pins these tactics instead of autotuning (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

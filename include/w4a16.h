@@ -373,20 +373,24 @@ int w4a16_get_tactic(int64_t M, int64_t N, int64_t K, int64_t G, int32_t* tactic
 /* Empties the tactic table. Always W4A16_OK. */
 int w4a16_clear_tactics(void);
 
-/* Times every valid tactic for the shape on the caller's buffers (A, Wt, S
- * read; C overwritten) on `stream`, `reps` launches each after one untimed
- * launch, and stores the fastest in the table (the page's timing cache).
- * With flush_dev (flush_bytes > 0; a device buffer larger than the L2 cache,
- * overwritten) every timed launch starts after the buffer is rewritten, so the
- * weights come from HBM as they do when many layers' weights stream by; with
- * flush_dev NULL the launches run back to back. Blocks the host until the
- * timing is done: call it at setup, not while the stream is being captured.
- * Writes the winning id to *best_tactic and its mean time per launch in
- * microseconds to *best_us (if not NULL). Same contract and errors as
- * w4a16_gemm, INVALID_ARG also for reps outside 1..10000. */
-int w4a16_autotune(const w4a16_half* A_dev, const uint8_t* Wt_dev, const w4a16_half* S_dev, w4a16_half* C_dev,
-                   int64_t M, int64_t N, int64_t K, int64_t G, int32_t reps, void* flush_dev,
-                   int64_t flush_bytes, int32_t* best_tactic, float* best_us, void* stream);
+/* Times every valid tactic for the shape and stores the fastest in the table
+ * (the page's timing cache). A [M, K] is read and C [M, N] overwritten; Wt and
+ * S are HOST arrays of `copies` device pointers to copies of the tiled weights
+ * and scales (1 <= copies <= 1024). For each tactic, `reps` launches rotating
+ * over the copies are recorded into a CUDA graph (on a stream of its own) and
+ * replayed on `stream`: launches back to back, as a model's layers run them,
+ * with their programmatic-dependent-launch overlap; when the copies together
+ * exceed the L2 cache the weights come from HBM, as they do when many layers'
+ * weights stream by. The time of a tactic is the fastest of three replays per
+ * launch. Blocks the host until the timing is done: call it at setup, not
+ * while `stream` is being captured. Writes the winning id to *best_tactic, its
+ * time per launch in microseconds to *best_us (if not NULL), and the time of
+ * tactic id t to times_us[t - 1] for the first times_capacity ids (times_us
+ * may be NULL when times_capacity is 0). Same contract and errors as
+ * w4a16_gemm; INVALID_ARG also for reps outside 1..10000. */
+int w4a16_autotune(const w4a16_half* A_dev, const uint8_t* const* Wt, const w4a16_half* const* S, int32_t copies,
+                   w4a16_half* C_dev, int64_t M, int64_t N, int64_t K, int64_t G, int32_t reps,
+                   int32_t* best_tactic, float* best_us, float* times_us, int32_t times_capacity, void* stream);
 
 /* Test aid for the failure path of the bounded device waits (no counterpart
  * on the plugin pages). For every later launch of the tensor-core GEMM kernel

@@ -234,13 +234,13 @@ def test_tactic_table_round_trip_on_host(lib):
 
 
 def test_autotune_rejects_bad_arguments_on_host(lib):
-    t = lambda **kw: w.w4a16_autotune(kw.get("A", FAKE), FAKE, FAKE, FAKE, kw.get("M", 4), 128, 128, 64,
-                                      reps=kw.get("reps", 5), flush=kw.get("flush"),
-                                      flush_bytes=kw.get("fb", 0), stream=0)[0]
+    t = lambda **kw: w.w4a16_autotune(kw.get("A", FAKE), kw.get("wts", [FAKE]), kw.get("ss", [FAKE]), FAKE,
+                                      kw.get("M", 4), 128, 128, 64, reps=kw.get("reps", 5), stream=0)[0]
     assert t(A=None) == w.ERR_INVALID_ARG
     assert t(M=0) == w.ERR_INVALID_ARG
     assert t(reps=0) == w.ERR_INVALID_ARG
-    assert t(fb=1024) == w.ERR_INVALID_ARG  # bytes to flush but no buffer
+    assert t(wts=[FAKE, 0], ss=[FAKE, FAKE]) == w.ERR_INVALID_ARG
+    assert t(wts=[FAKE + 8]) == w.ERR_MISALIGNED
     assert t(A=FAKE + 8) == w.ERR_MISALIGNED
     try:
         import torch

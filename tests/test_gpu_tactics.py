@@ -57,18 +57,19 @@ def test_every_tactic_matches_the_oracle(o, M, K, N, G):
     assert w.device_status() == w.OK
 
 
-@pytest.mark.parametrize("flush", [False, True])
-def test_autotune_stores_the_fastest_and_the_gemm_uses_it(o, flush):
+@pytest.mark.parametrize("copies", [1, 3])
+def test_autotune_stores_the_fastest_and_the_gemm_uses_it(o, copies):
     M, K, N, G = 16, 4096, 4096, 128
     c = workloads.dense(M, K, N, G, seed=33)
     _, wt = device_weights(c.q)
     A, S = dev(c.A), dev(c.S)
     C = torch.empty((M, N), dtype=torch.float16, device="cuda")
-    fl = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if flush else None
-    rc, best, us = w.w4a16_autotune(A, wt, S, C, M, N, K, G, reps=5, flush=fl)
+    wts, Ss = [wt] + [wt.clone() for _ in range(copies - 1)], [S] + [S.clone() for _ in range(copies - 1)]
+    rc, best, us, times = w.w4a16_autotune(A, wts, Ss, C, M, N, K, G, reps=8, with_times=True)
     assert rc == w.OK
     _, ids = w.w4a16_get_valid_tactics(M, N, K, G)
-    assert best in ids and 0 < us < 1e4
+    assert best in ids and 0 < us < 1e4 and len(times) == len(ids)
+    assert us == pytest.approx(min(times)) and all(x > 0 for x in times)
     assert w.w4a16_get_tactic(M, N, K, G) == best
     assert w.w4a16_gemm_launch_info(M, N, K, G)[1].as_dict() == w.w4a16_tactic_launch_info(M, N, K, G, best)[1].as_dict()
     got = w.gemm(A, wt, S, N, G).cpu().numpy()

@@ -139,8 +139,9 @@ def load() -> ctypes.CDLL:
         lib.w4a16_get_tactic.restype = ctypes.c_int
         lib.w4a16_clear_tactics.argtypes = []
         lib.w4a16_clear_tactics.restype = ctypes.c_int
-        lib.w4a16_autotune.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.c_int32, _vp, _i64, _i32p,
-                                       ctypes.POINTER(ctypes.c_float), _vp]
+        lib.w4a16_autotune.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.c_int32, _vp, _i64, _i64,
+                                       _i64, _i64, ctypes.c_int32, _i32p, ctypes.POINTER(ctypes.c_float),
+                                       ctypes.POINTER(ctypes.c_float), ctypes.c_int32, _vp]
         lib.w4a16_autotune.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -286,15 +287,18 @@ def w4a16_clear_tactics() -> int:
     return load().w4a16_clear_tactics()
 
 
-def w4a16_autotune(A, Wt, S, C, M: int, N: int, K: int, G: int, reps: int = 20, flush=None, flush_bytes: int = 0,
-                   stream=None):
-    """(status, best tactic id, its mean microseconds per launch)."""
+def w4a16_autotune(A, Wts: Sequence, Ss: Sequence, C, M: int, N: int, K: int, G: int, reps: int = 20,
+                   stream=None, with_times: bool = False):
+    """Times every tactic over the weight copies Wts / Ss (rotating); (status, best tactic id,
+    its microseconds per launch[, microseconds of every tactic])."""
     best = ctypes.c_int32(0)
     us = ctypes.c_float(0.0)
-    if flush is not None and not flush_bytes:
-        flush_bytes = flush.numel() * flush.element_size()
-    rc = load().w4a16_autotune(_addr(A), _addr(Wt), _addr(S), _addr(C), M, N, K, G, reps, _addr(flush), flush_bytes,
-                               ctypes.byref(best), ctypes.byref(us), _stream(stream))
+    times = (ctypes.c_float * 64)()
+    rc = load().w4a16_autotune(_addr(A), _ptr_array(Wts), _ptr_array(Ss), len(Wts), _addr(C), M, N, K, G, reps,
+                               ctypes.byref(best), ctypes.byref(us), times, 64, _stream(stream))
+    if with_times:
+        n = len(w4a16_get_valid_tactics(M, N, K, G)[1])
+        return rc, best.value, us.value, [times[i] for i in range(min(n, 64))]
     return rc, best.value, us.value
 
 
