@@ -86,6 +86,8 @@ class Oracle:
         lib.oracle_tile_w8.restype = None
         lib.oracle_gemm_w8.argtypes = [_u16p, _i8p, _u16p, _i64, _i64, _i64, _i64, _u16p, ctypes.c_int]
         lib.oracle_gemm_w8.restype = ctypes.c_int
+        lib.oracle_quantize_w8.argtypes = [_u16p, _i64, _i64, _i64, _i8p, _u16p]
+        lib.oracle_quantize_w8.restype = None
         lib.oracle_threads.restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -206,6 +208,15 @@ class Oracle:
         if rc:
             raise RuntimeError(f"oracle_gemm_w8 failed ({rc})")
         return c.view(np.float16)
+
+    def quantize_w8(self, W: np.ndarray, G: int):
+        """Group-wise 8-bit quantisation of fp16 W [K, N]: (int8 codes [K, N], fp16 scales)."""
+        w = _bits(W)
+        K, N = w.shape
+        q8 = np.zeros((K, N), dtype=np.int8)
+        S = np.zeros(((K + G - 1) // G, N), dtype=np.uint16)
+        self.lib.oracle_quantize_w8(_ptr(w, _u16p), K, N, G, _ptr(q8, _i8p), _ptr(S, _u16p))
+        return q8, S.view(np.float16)
 
     def quantize(self, W: np.ndarray, G: int):
         """Group-wise int4 quantisation of fp16 W [K, N]: (canonical packed codes, fp16 scales)."""

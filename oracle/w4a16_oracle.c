@@ -464,3 +464,52 @@ int oracle_gemm_w8(const uint16_t* A, const int8_t* q8, const uint16_t* S, int64
     free(a);
     return failed ? 2 : 0;
 }
+
+/*
+ * Group-wise symmetric 8-bit quantisation of fp16 weights W [K, N] (the export
+ * step of the W8A16 variant): the KV Cache INT8 quantization page's symmetric
+ * rule (scale = max|x| / 127, x_q = round(x / scale), in float) over each group
+ * of G rows of one column, the scale stored in fp16:
+ *   s[g, n] = fp16_rne( float(amax) / 127.0f )
+ *   q8[k, n] = clamp( round(float(W[k, n]) / float(s[g, n])), -128, 127 ),
+ *              q8 = 0 where s = 0
+ * round() takes halves away from zero. Codes are written one per byte, q8
+ * [K, N] row-major; the scales as fp16 bits. W must be finite.
+ */
+void oracle_quantize_w8(const uint16_t* W, int64_t K, int64_t N, int64_t G, int8_t* q8, uint16_t* S) {
+    const int64_t groups = (K + G - 1) / G;
+    for (int64_t g = 0; g < groups; ++g) {
+        const int64_t k0 = g * G;
+        const int64_t k1 = k0 + G < K ? k0 + G : K;
+        for (int64_t n = 0; n < N; ++n) {
+            float amax = 0.0f;
+            for (int64_t k = k0; k < k1; ++k) {
+                float a = fabsf((float)oracle_half_to_double(W[k * N + n]));
+                if (a > amax) amax = a;
+            }
+#if ORACLE_MUTANT == 18
+            float s32 = amax / 128.0f; /* the 8-bit range taken as 128 */
+#else
+            float s32 = amax / 127.0f;
+#endif
+            uint16_t sh = oracle_double_to_half((double)s32);
+            S[g * N + n] = sh;
+            float s = (float)oracle_half_to_double(sh);
+            for (int64_t k = k0; k < k1; ++k) {
+                int q = 0;
+                if (s != 0.0f) {
+                    float x = (float)oracle_half_to_double(W[k * N + n]) / s;
+#if ORACLE_MUTANT == 19
+                    float r = nearbyintf(x); /* halves to even */
+#else
+                    float r = roundf(x);
+#endif
+                    q = (int)r;
+                    if (q < -128) q = -128;
+                    if (q > 127) q = 127;
+                }
+                q8[k * N + n] = (int8_t)q;
+            }
+        }
+    }
+}

@@ -324,8 +324,8 @@ def pin_sample_matches_full(o) -> bool:
     return bool(np.array_equal(got.view(np.uint16), full[rows, cols].view(np.uint16)))
 
 
-def _read_quantize_example():
-    path = os.path.join(GOLDEN, "quantize_example.txt")
+def _read_quantize_example(name="quantize_example.txt"):
+    path = os.path.join(GOLDEN, name)
     sections, cur, dims = {}, None, {}
     with open(path) as f:
         for line in f:
@@ -517,10 +517,41 @@ def pin_w8_numpy_blas(o) -> bool:
     return bool(np.all(np.abs(got - ref.view(np.uint16).astype(np.int32)) <= 1))
 
 
+def pin_quantize_w8_golden(o) -> bool:
+    """The hand-worked 8-bit example: scales bit for bit (one just above the smallest normal
+    fp16), codes exactly (an exact half rounds away from zero, an all-zero group gives 0)."""
+    dims, t = _read_quantize_example("quantize_w8_example.txt")
+    W = t["W"].astype(np.float16)
+    q8, S = o.quantize_w8(W, dims["G"])
+    return (bool(np.array_equal(S.view(np.uint16), t["S"].astype(np.float16).view(np.uint16)))
+            and bool(np.array_equal(q8, t["Q"].astype(np.int8))))
+
+
+def pin_quantize_w8_properties(o) -> bool:
+    """Random weights: codes within [-127, 127]; each group's largest |w| gets +-127; every
+    code reconstructs its weight within half a scale step; 2W gives 2s and the same codes."""
+    W, K, N, G = _quantize_case(seed=24)
+    q8, S = o.quantize_w8(W, G)
+    s = S.astype(np.float64)[np.arange(K) // G]
+    w = W.astype(np.float64)
+    if q8.min() < -127 or q8.max() > 127:
+        return False
+    if np.any(np.abs(q8 * s - w) > s / 2 * (1 + 1e-6)):
+        return False
+    for g in range(-(-K // G)):
+        rows = slice(g * G, min(K, (g + 1) * G))
+        top = np.argmax(np.abs(w[rows]), axis=0)
+        if not np.all(np.abs(q8[rows][top, np.arange(N)]) == 127):
+            return False
+    q2, S2 = o.quantize_w8((2 * W.astype(np.float32)).astype(np.float16), G)
+    return bool(np.array_equal(q2, q8)) and bool(np.array_equal(S2.astype(np.float64), 2 * S.astype(np.float64)))
+
+
 PINS = [pin_half_widening, pin_half_rounding, pin_half_rounding_numpy, pin_pack_golden,
         pin_pack_all_bytes, pin_pack_random_odd_k, pin_tiled_positions, pin_tiled_roundtrip,
         pin_exact_small, pin_near_ties, pin_closed_form, pin_one_hot, pin_scale_duplication,
         pin_numpy_blas, pin_grouped_segments, pin_grouped_brute, pin_sample_matches_full,
         pin_quantize_golden, pin_quantize_properties, pin_quantize_scale_invariance,
         pin_quantize_groups_independent, pin_quantize_edges, pin_w8_tiled_positions, pin_w8_tiled_roundtrip,
-        pin_w8_exact_small, pin_w8_closed_form, pin_w8_one_hot, pin_w8_numpy_blas]
+        pin_w8_exact_small, pin_w8_closed_form, pin_w8_one_hot, pin_w8_numpy_blas, pin_quantize_w8_golden,
+        pin_quantize_w8_properties]

@@ -42,6 +42,8 @@ MUTANTS = {
     15: "quantiser scale from the whole column",
     16: "8-bit codes read as unsigned",
     17: "8-bit tiled layout with the bytes of a chunk reversed",
+    18: "8-bit quantiser scale taken as max/128",
+    19: "8-bit quantiser rounds halves to even",
 }
 
 
