@@ -403,32 +403,26 @@ def run_ours(args):
     if status != w4.OK:
         raise RuntimeError(f"device status after the timed region: {w4.status_string(status)}")
 
-    # End to end through the public API: pinned host activations in, results out, every step.
-    # The step's two inputs (1 and 16 rows) travel in one 17-row buffer and its two
-    # outputs come back in one, so each step makes one copy each way.
-    A_h = torch.from_numpy(np.concatenate([case.A[:1], case.A], axis=0)).pin_memory()
-    C_h = torch.empty((1 + 16, N_DIM), dtype=torch.float16).pin_memory()
-    A_d = torch.empty((1 + 16, K_DIM), dtype=torch.float16, device=dev)
-    C_d = torch.empty((1 + 16, N_DIM), dtype=torch.float16, device=dev)
-    A1_d, A16_d = A_d[:1], A_d[1:]
-    C1_d, C16_d = C_d[:1], C_d[1:]
-    K_e2e = min(K, 2000)
-
-    # The steps as a server runs independent batches: each step copies its
-    # activations in from pinned host memory, runs the two GEMMs through the C
-    # entry point and copies both results out to pinned host memory. The copies
-    # run on two more streams (one per direction, so the two copy engines work at
-    # once) into double buffers, so that step i's GEMMs overlap the copy-in of
-    # step i+1 and the copy-out of step i-1. E2E_GRAPH_STEPS steps
-    # (rotating weight copies as in the timed region) are recorded once into a
-    # CUDA graph and replayed; every step still moves its inputs in and its
-    # outputs out.
-    E2E_GRAPH_STEPS = 16
+    # End to end through the public C entry point, as a server runs independent
+    # batches: every step's activations (1 + 16 rows) come in from pinned host
+    # memory and both results go back out to pinned host memory. The copies move
+    # E2E_BATCH steps' inputs (or outputs) at a time, on one stream per direction
+    # (the two copy engines work at once), into double batch buffers, so that a
+    # batch's GEMMs overlap the next batch's copy-in and the previous batch's
+    # copy-out. (A copy on another stream that a GEMM must wait for takes that
+    # GEMM out of the programmatic-dependent-launch overlap with the kernel before
+    # it; per-step copies cost about 4 us per step that way.) E2E_GRAPH_STEPS
+    # steps, rotating weight copies as in the timed region, are recorded once
+    # into a CUDA graph and replayed.
+    E2E_BATCH, E2E_GRAPH_STEPS = 8, 32
+    rows_step = 1 + 16
+    A_step = np.concatenate([case.A[:1], case.A], axis=0)
+    A_h = torch.from_numpy(np.concatenate([A_step] * E2E_BATCH, axis=0)).pin_memory()
+    C_h = torch.empty((E2E_BATCH * rows_step, N_DIM), dtype=torch.float16).pin_memory()
+    A_db = [torch.empty((E2E_BATCH * rows_step, K_DIM), dtype=torch.float16, device=dev) for _ in range(2)]
+    C_db = [torch.empty((E2E_BATCH * rows_step, N_DIM), dtype=torch.float16, device=dev) for _ in range(2)]
+    K_e2e = min(K, 2048)
     cgemm = w4.load().w4a16_gemm
-    A_db = [A_d, torch.empty_like(A_d)]
-    C_db = [C_d, torch.empty_like(C_d)]
-    a_ptr = [(x[:1].data_ptr(), x[1:].data_ptr()) for x in A_db]
-    c_ptr = [(x[:1].data_ptr(), x[1:].data_ptr()) for x in C_db]
     wptr = [x.data_ptr() for x in wts]
     sptr = [x.data_ptr() for x in Ss]
     in_stream, out_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)  # one copy engine per direction
@@ -436,36 +430,42 @@ def run_ours(args):
     def e2e_steps(n):
         comp = torch.cuda.current_stream(dev)
         st = comp.cuda_stream
-        ev_in = [torch.cuda.Event() for _ in range(n)]
-        ev_out = [torch.cuda.Event() for _ in range(n)]
-        ev_back = [torch.cuda.Event() for _ in range(n)]
+        nb = n // E2E_BATCH
+        ev_in = [torch.cuda.Event() for _ in range(nb)]
+        ev_out = [torch.cuda.Event() for _ in range(nb)]
+        ev_back = [torch.cuda.Event() for _ in range(nb)]
         in_stream.wait_stream(comp)
         out_stream.wait_stream(comp)
 
-        def copy_in(i):
+        def copy_in(j):
             with torch.cuda.stream(in_stream):
-                if i >= 2:
-                    in_stream.wait_event(ev_out[i - 2])  # step i-2's GEMMs have read this buffer
-                A_db[i % 2].copy_(A_h, non_blocking=True)
-                ev_in[i].record(in_stream)
+                if j >= 2:
+                    in_stream.wait_event(ev_out[j - 2])  # batch j-2's GEMMs have read this buffer
+                A_db[j % 2].copy_(A_h, non_blocking=True)
+                ev_in[j].record(in_stream)
 
         copy_in(0)
-        for i in range(n):
-            b = i % 2
-            if i + 1 < n:
-                copy_in(i + 1)
-            comp.wait_event(ev_in[i])
-            if i >= 2:
-                comp.wait_event(ev_back[i - 2])  # step i-2's results have left this buffer
-            r1, r2 = (2 * i) % R, (2 * i + 1) % R
-            if cgemm(a_ptr[b][0], wptr[r1], sptr[r1], c_ptr[b][0], 1, N_DIM, K_DIM, G_DIM, st) or \
-                    cgemm(a_ptr[b][1], wptr[r2], sptr[r2], c_ptr[b][1], 16, N_DIM, K_DIM, G_DIM, st):
-                raise RuntimeError("a GEMM call failed in the end-to-end loop")
-            ev_out[i].record(comp)
+        for j in range(nb):
+            b = j % 2
+            if j + 1 < nb:
+                copy_in(j + 1)
+            comp.wait_event(ev_in[j])
+            if j >= 2:
+                comp.wait_event(ev_back[j - 2])  # batch j-2's results have left this buffer
+            for u in range(E2E_BATCH):
+                i = j * E2E_BATCH + u
+                a0 = A_db[b][u * rows_step:(u + 1) * rows_step]
+                c0 = C_db[b][u * rows_step:(u + 1) * rows_step]
+                r1, r2 = (2 * i) % R, (2 * i + 1) % R
+                if cgemm(a0[:1].data_ptr(), wptr[r1], sptr[r1], c0[:1].data_ptr(), 1, N_DIM, K_DIM, G_DIM, st) or \
+                        cgemm(a0[1:].data_ptr(), wptr[r2], sptr[r2], c0[1:].data_ptr(), 16, N_DIM, K_DIM, G_DIM,
+                              st):
+                    raise RuntimeError("a GEMM call failed in the end-to-end loop")
+            ev_out[j].record(comp)
             with torch.cuda.stream(out_stream):
-                out_stream.wait_event(ev_out[i])
+                out_stream.wait_event(ev_out[j])
                 C_h.copy_(C_db[b], non_blocking=True)
-                ev_back[i].record(out_stream)
+                ev_back[j].record(out_stream)
         comp.wait_stream(in_stream)
         comp.wait_stream(out_stream)
 
@@ -491,9 +491,10 @@ def run_ours(args):
     e2e = {"value": job_throughput(K_e2e * step_bytes(), world, e2e_sec) / 1e9, "unit": "GB/s",
            "h2d_bytes_per_step": sum(m * K_DIM * 2 for m in M_STEP),
            "d2h_bytes_per_step": sum(m * N_DIM * 2 for m in M_STEP), "steps": K_e2e,
-           "launch": f"CUDA graph of {E2E_GRAPH_STEPS} steps, replayed: per step one copy in (pinned host -> device), "
-                     "two w4a16_gemm calls, one copy out (device -> pinned host); copies on one stream per "
-                     "direction with double buffers overlap the neighbouring steps' GEMMs"}
+           "launch": f"CUDA graph of {E2E_GRAPH_STEPS} steps, replayed: every step's inputs copied in from "
+                     f"pinned host memory and its outputs copied out, {E2E_BATCH} steps per copy, on one stream "
+                     "per direction with double batch buffers overlapping the neighbouring batches' GEMMs; two "
+                     "w4a16_gemm calls per step"}
 
     extra = per_config(w4, dev, tune=not args.no_tune) if (rank == 0 and not args.no_configs) else None
     tactics = tactic_report(w4, dev) if (rank == 0 and not args.no_configs) else None
@@ -722,29 +723,32 @@ def per_config(w4, dev, tune=True):
             out[name]["tactic"] = tactic
         del g
     out["quantize"] = quantize_timing(w4, dev, peaks, l2)
+    out["quantize_w8"] = quantize_timing(w4, dev, peaks, l2, bits=8)
     status = w4.device_status(clear=True)
     if status != w4.OK:
         raise RuntimeError(f"device status after per-config timing: {w4.status_string(status)}")
     return out
 
 
-def quantize_timing(w4, dev, peaks, l2, K=4096, N=14336, G=128):
+def quantize_timing(w4, dev, peaks, l2, K=4096, N=14336, G=128, bits=4):
     """The export-time quantiser (setup, not on the GEMM path) on the MLP up projection's
-    fp16 weights: W read once, packed codes and scales written once per launch."""
+    fp16 weights: W read once, codes (int4 packed, or 8-bit) and scales written once per launch."""
     import torch
     gen = torch.Generator(device=dev).manual_seed(5)
     per_w = K * N * 2
-    by = per_w + ((K + 1) // 2) * N + ((K + G - 1) // G) * N * 2
+    code_bytes = ((K + 1) // 2) * N if bits == 4 else K * N
+    by = per_w + code_bytes + ((K + G - 1) // G) * N * 2
     R = max(2, math.ceil(2 * l2 / per_w) + 1)
     sets = []
     for _ in range(R):
         W = (torch.randn((K, N), generator=gen, device=dev, dtype=torch.float32) * 0.02).half()
-        sets.append((W, torch.empty(((K + 1) // 2, N), dtype=torch.uint8, device=dev),
-                     torch.empty(((K + G - 1) // G, N), dtype=torch.float16, device=dev)))
+        codes = (torch.empty(((K + 1) // 2, N), dtype=torch.uint8, device=dev) if bits == 4
+                 else torch.empty((K, N), dtype=torch.int8, device=dev))
+        sets.append((W, codes, torch.empty(((K + G - 1) // G, N), dtype=torch.float16, device=dev)))
 
     def launch(r):
         W, wp, S = sets[r]
-        rc = w4.w4a16_quantize(W, wp, S, K, N, G)
+        rc = (w4.w4a16_quantize if bits == 4 else w4.w8a16_quantize)(W, wp, S, K, N, G)
         if rc:
             raise RuntimeError(w4.status_string(rc))
     launch(0)

@@ -142,6 +142,19 @@ int w4a16_repack(const uint8_t* wp_dev, uint8_t* wt_dev, int64_t K, int64_t N, v
 int w4a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt_dev, const w4a16_half* S_dev,
                w4a16_half* C_dev, int64_t M, int64_t N, int64_t K, int64_t G, void* stream);
 
+/* Flags of w4a16_gemm_ex. */
+#define W4A16_FLAG_STATIC_WEIGHTS 1u /* this call's Wt and S are not written by any kernel that may still be
+                                        running on the stream (weights prepared at load time): the GEMM may
+                                        stream them before the previous kernel on the stream finishes */
+
+/* w4a16_gemm with per-call flags (0 or W4A16_FLAG_STATIC_WEIGHTS): the
+ * static-weights promise of w4a16_set_static_weights scoped to this one call,
+ * so that one stream's GEMMs can stream their fixed weights early while
+ * another stream repacks or requantises others. Same contract and errors as
+ * w4a16_gemm; INVALID_ARG also for unknown flag bits. */
+int w4a16_gemm_ex(const w4a16_half* A_dev, const uint8_t* Wt_dev, const w4a16_half* S_dev, w4a16_half* C_dev,
+                  int64_t M, int64_t N, int64_t K, int64_t G, uint32_t flags, void* stream);
+
 /* Grouped-expert form. A_dev [total_rows, K] holds the activation rows
  * already gathered per expert; rows [off[e], off[e+1]) of A_dev and of
  * C_dev [total_rows, N] belong to expert e, which uses tiled weights
@@ -317,6 +330,19 @@ int w4a16_grouped_launch_info(int64_t E, int64_t total_rows, int64_t N, int64_t 
  * holding k_local 16h + b as a two's-complement byte; rows k >= K and columns
  * n >= N hold 0. The product runs on the tensor-core kernel for every M.
  * ------------------------------------------------------------------------- */
+
+/* Group-wise symmetric 8-bit quantisation of fp16 weights W_dev [K, N], the
+ * export step of W8A16: the KV Cache INT8 quantization page's symmetric rule
+ * (scale = max|x| / 127, x_q = round(x / scale)) over each group of G rows of
+ * one column, the scale kept in fp16:
+ *     s[g, n] = fp16_rne(float(max |W[k, n]| over group g) / 127)
+ *     q8[k, n] = clamp(round(float(W[k, n]) / float(s[g, n])), -128, 127)
+ * with IEEE float division and halves rounded away from zero; q8 = 0 where
+ * s = 0. Codes to q8_dev [K, N] int8 row-major, scales to S_dev [ceil(K/G), N].
+ * Same contract, alignment and errors as w4a16_quantize (q8_dev 2-byte
+ * aligned). */
+int w8a16_quantize(const w4a16_half* W_dev, int8_t* q8_dev, w4a16_half* S_dev, int64_t K, int64_t N, int64_t G,
+                   void* stream);
 
 /* Size in bytes of the 8-bit tiled layout for K x N codes (0 if K or N <= 0). */
 int64_t w8a16_tiled_bytes(int64_t K, int64_t N);

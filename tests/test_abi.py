@@ -198,7 +198,7 @@ def test_tactic_lists_on_host(lib):
     # Decode shape: the skinny forms (K split 1..8, one or two K halves, two ring
     # depths) first, then the tensor-core forms (token tiles 16..256, K split 1/2/4/8).
     rc, ids = w.w4a16_get_valid_tactics(1, 4096, 4096, 128)
-    assert rc == w.OK and ids == list(range(1, len(ids) + 1)) and 32 < len(ids) <= 64
+    assert rc == w.OK and ids == list(range(1, len(ids) + 1)) and 32 < len(ids) <= 96
     infos = [w.w4a16_tactic_launch_info(1, 4096, 4096, 128, t) for t in ids]
     assert all(rc == w.OK for rc, _ in infos)
     kinds = [i.threads_per_cta in (256, 512) and i.token_tile == 8 for _, i in infos]
@@ -276,3 +276,18 @@ def test_static_scratch_layer_host_checks(lib):
     assert call(512, 4096, 14336) == w.ERR_SCRATCH_TOO_SMALL
     assert call(4, 4096, 0) == w.ERR_INVALID_ARG
     assert call(0, 4096, 14336) == w.OK
+
+
+def test_gemm_ex_flags_on_host(lib):
+    g = lambda flags, M=4: w.w4a16_gemm_ex(FAKE, FAKE, FAKE, FAKE, M, 128, 128, 64, flags, stream=0)
+    assert g(2) == w.ERR_INVALID_ARG and g(0x80000000) == w.ERR_INVALID_ARG
+    assert g(w.FLAG_STATIC_WEIGHTS, M=0) == w.OK and g(0, M=0) == w.OK
+    assert g(w.FLAG_STATIC_WEIGHTS, M=-1) == w.ERR_INVALID_ARG
+
+
+def test_w8_quantize_rejects_bad_arguments_on_host(lib):
+    q = lambda **kw: w.w8a16_quantize(kw.get("W", FAKE), kw.get("q8", FAKE), kw.get("S", FAKE), kw.get("K", 64),
+                                      kw.get("N", 64), kw.get("G", 32), stream=0)
+    assert q(W=None) == w.ERR_INVALID_ARG and q(K=0) == w.ERR_INVALID_ARG
+    assert q(N=63) == w.ERR_UNSUPPORTED and q(G=33) == w.ERR_UNSUPPORTED
+    assert q(W=FAKE + 2) == w.ERR_MISALIGNED and q(q8=FAKE + 1) == w.ERR_MISALIGNED

@@ -347,6 +347,28 @@ def test_static_weights_mode(o):
             assert ok, f"static weights, case {idx}: max abs err {err}"
 
 
+def test_static_weights_per_call(o):
+    # The same promise scoped to single calls (w4a16_gemm_ex): calls with and without
+    # the flag interleaved on one stream, the process-wide setting left off.
+    assert w.w4a16_set_static_weights(False) == 0
+    cases = [workloads.make("decode_m1"), workloads.dense(40, 1024, 640, 64, 55)]
+    prepared = [(c, device_weights(c.q)[1], dev(c.A), dev(c.S)) for c in cases]
+    torch.cuda.synchronize()
+    outs = []
+    for c, wt, A, S in prepared:
+        for flags in (w.FLAG_STATIC_WEIGHTS, 0, w.FLAG_STATIC_WEIGHTS):
+            C = torch.empty((c.M, c.N), dtype=torch.float16, device="cuda")
+            assert w.w4a16_gemm_ex(A, wt, S, C, c.M, c.N, c.K, c.G, flags) == w.OK
+            outs.append(C)
+    torch.cuda.synchronize()
+    assert w.w4a16_set_static_weights(False) == 0  # the call scope did not leak into the global setting
+    for idx, (c, _, _, _) in enumerate(prepared):
+        ref = o.gemm(c.A, pins.python_pack(c.q), c.S, c.K, c.G)
+        for got in outs[3 * idx:3 * idx + 3]:
+            ok, err, rel = within_tolerance(got.cpu().numpy(), ref)
+            assert ok, f"per-call static weights, case {idx}: max abs err {err}"
+
+
 def test_repack_then_gemm_back_to_back(o):
     # The GEMM right after the repack kernel that produced its weights, on one stream.
     for c in (workloads.dense(8, 4096, 14336, 128, 53), workloads.dense(16, 14336, 1024, 128, 54)):

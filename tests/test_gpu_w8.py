@@ -56,3 +56,29 @@ def test_w8_gemm_matches_oracle(o, M, K, N, G):
 @pytest.mark.parametrize("name", ["w8_decode_m16", "w8_prefill"])
 def test_w8_full_size(o, name):
     run_w8(o, workloads.make(name))
+
+
+@pytest.mark.parametrize("K,N,G", [(192, 256, 64), (131, 264, 64), (300, 40, 128), (4096, 1024, 128), (64, 520, 256)])
+def test_w8_quantize_bit_exact(o, K, N, G):
+    # staged (N % 8 == 0, G <= 256) and fallback forms, odd K and a partial last group
+    g = np.random.Generator(np.random.PCG64(K * 7 + N))
+    W = (g.standard_normal((K, N)) * g.uniform(0.005, 2.0, size=(1, N))).astype(np.float16)
+    q8, S = w.quantize_w8(dev(W), G)
+    torch.cuda.synchronize()
+    ref_q, ref_S = o.quantize_w8(W, G)
+    assert np.array_equal(S.cpu().numpy().view(np.uint16), ref_S.view(np.uint16))
+    assert np.array_equal(q8.cpu().numpy(), ref_q)
+    assert w.device_status() == w.OK
+
+
+def test_w8_quantize_then_gemm(o):
+    # the export chain: fp16 weights -> 8-bit codes and scales -> tiled layout -> product
+    M, K, N, G = 24, 1024, 512, 128
+    g = np.random.Generator(np.random.PCG64(77))
+    W = (g.standard_normal((K, N)) * 0.02).astype(np.float16)
+    A = g.standard_normal((M, K), dtype=np.float32).astype(np.float16)
+    q8, S = w.quantize_w8(dev(W), G)
+    C = w.gemm_w8(dev(A), w.repack_w8(q8), S, N, G).cpu().numpy()
+    ref_q, ref_S = o.quantize_w8(W, G)
+    ok, err, _ = within_tolerance(C, o.gemm_w8(A, ref_q, ref_S, K, G))
+    assert ok, err

@@ -12,6 +12,7 @@ from ._lib import (  # noqa: F401
     w4a16_set_static_weights, w4a16_tiled_bytes, w4a16_unpack, w4a16_get_valid_tactics, w4a16_tactic_launch_info,
     w4a16_set_tactic, w4a16_get_tactic, w4a16_clear_tactics, w4a16_autotune, w8a16_tiled_bytes, w8a16_repack,
     w8a16_gemm, w8a16_gemm_launch_info, repack_w8, gemm_w8, w4a16_moe_layer_static, w4a16_moe_static_scratch_bytes,
+    w4a16_gemm_ex, FLAG_STATIC_WEIGHTS, w8a16_quantize, quantize_w8,
 )
 from ._lib import (  # noqa: F401
     ACT_GELU_ERF, ACT_GELU_TANH, ACT_IDENTITY, ACT_RELU, ERR_BAD_OFFSETS, ERR_BAD_ROUTING, ERR_CUDA,

@@ -27,6 +27,7 @@ ERR_BAD_ROUTING = 7
 ERR_SCRATCH_TOO_SMALL = 8
 MAX_EXPERTS = 64
 MAX_TOPK = 8
+FLAG_STATIC_WEIGHTS = 1
 ACT_IDENTITY = 0
 ACT_RELU = 1
 ACT_GELU_ERF = 2
@@ -40,7 +41,7 @@ EXPORTED = [
     "w4a16_moe_workspace_size", "w4a16_moe_layer", "w4a16_get_valid_tactics", "w4a16_tactic_launch_info",
     "w4a16_set_tactic", "w4a16_get_tactic", "w4a16_clear_tactics", "w4a16_autotune",
     "w8a16_tiled_bytes", "w8a16_repack", "w8a16_gemm", "w8a16_gemm_launch_info",
-    "w4a16_moe_layer_static", "w4a16_moe_static_scratch_bytes",
+    "w4a16_moe_layer_static", "w4a16_moe_static_scratch_bytes", "w4a16_gemm_ex", "w8a16_quantize",
 ]
 
 
@@ -84,6 +85,8 @@ def load() -> ctypes.CDLL:
         lib.w4a16_tiled_bytes.restype = _i64
         lib.w4a16_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]
         lib.w4a16_gemm.restype = ctypes.c_int
+        lib.w4a16_gemm_ex.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.c_uint32, _vp]
+        lib.w4a16_gemm_ex.restype = ctypes.c_int
         lib.w4a16_grouped_gemm.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _vp, _i64, _i64,
                                            _i64, _i64, _i64, _vp]
         lib.w4a16_grouped_gemm.restype = ctypes.c_int
@@ -120,6 +123,8 @@ def load() -> ctypes.CDLL:
         lib.w4a16_moe_layer_static.restype = ctypes.c_int
         lib.w4a16_moe_static_scratch_bytes.argtypes = []
         lib.w4a16_moe_static_scratch_bytes.restype = _i64
+        lib.w8a16_quantize.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp]
+        lib.w8a16_quantize.restype = ctypes.c_int
         lib.w8a16_tiled_bytes.argtypes = [_i64, _i64]
         lib.w8a16_tiled_bytes.restype = _i64
         lib.w8a16_repack.argtypes = [_vp, _vp, _i64, _i64, _vp]
@@ -210,6 +215,10 @@ def w4a16_gemm(A, Wt, S, C, M: int, N: int, K: int, G: int, stream=None) -> int:
     return load().w4a16_gemm(_addr(A), _addr(Wt), _addr(S), _addr(C), M, N, K, G, _stream(stream))
 
 
+def w4a16_gemm_ex(A, Wt, S, C, M: int, N: int, K: int, G: int, flags: int, stream=None) -> int:
+    return load().w4a16_gemm_ex(_addr(A), _addr(Wt), _addr(S), _addr(C), M, N, K, G, flags, _stream(stream))
+
+
 def w4a16_grouped_gemm(A, Wt: Sequence, S: Sequence, offsets, C, E: int, total_rows: int, N: int, K: int,
                        G: int, stream=None) -> int:
     wt_arr = (_vp * max(1, len(Wt)))(*[_addr(w) for w in Wt])
@@ -261,9 +270,9 @@ def w4a16_moe_layer(X, logits, Wt_up: Sequence, S_up: Sequence, Wt_down: Sequenc
 def w4a16_get_valid_tactics(M: int, N: int, K: int, G: int):
     """(status, [tactic ids]) for a shape."""
     count = ctypes.c_int32(0)
-    arr = (ctypes.c_int32 * 64)()
-    rc = load().w4a16_get_valid_tactics(M, N, K, G, arr, 64, ctypes.byref(count))
-    return rc, [arr[i] for i in range(min(count.value, 64))]
+    arr = (ctypes.c_int32 * 96)()
+    rc = load().w4a16_get_valid_tactics(M, N, K, G, arr, 96, ctypes.byref(count))
+    return rc, [arr[i] for i in range(min(count.value, 96))]
 
 
 def w4a16_tactic_launch_info(M: int, N: int, K: int, G: int, tactic: int):
@@ -293,13 +302,17 @@ def w4a16_autotune(A, Wts: Sequence, Ss: Sequence, C, M: int, N: int, K: int, G:
     its microseconds per launch[, microseconds of every tactic])."""
     best = ctypes.c_int32(0)
     us = ctypes.c_float(0.0)
-    times = (ctypes.c_float * 64)()
+    times = (ctypes.c_float * 96)()
     rc = load().w4a16_autotune(_addr(A), _ptr_array(Wts), _ptr_array(Ss), len(Wts), _addr(C), M, N, K, G, reps,
-                               ctypes.byref(best), ctypes.byref(us), times, 64, _stream(stream))
+                               ctypes.byref(best), ctypes.byref(us), times, 96, _stream(stream))
     if with_times:
         n = len(w4a16_get_valid_tactics(M, N, K, G)[1])
-        return rc, best.value, us.value, [times[i] for i in range(min(n, 64))]
+        return rc, best.value, us.value, [times[i] for i in range(min(n, 96))]
     return rc, best.value, us.value
+
+
+def w8a16_quantize(W, q8, S, K: int, N: int, G: int, stream=None) -> int:
+    return load().w8a16_quantize(_addr(W), _addr(q8), _addr(S), K, N, G, _stream(stream))
 
 
 def w8a16_tiled_bytes(K: int, N: int) -> int:
@@ -467,6 +480,20 @@ def moe_layer(X, logits, wts_up: Sequence, Ss_up: Sequence, wts_down: Sequence, 
                            list(wts_down), [s.contiguous() for s in Ss_down], C, T, E, top_k, H, I, G, act,
                            workspace, workspace.numel(), stream), "w4a16_moe_layer")
     return C
+
+
+def quantize_w8(W, G: int, stream=None):
+    """fp16 weights [K, N] (device) -> (int8 codes [K, N], fp16 scales [ceil(K/G), N]): group-wise
+    symmetric 8-bit quantisation."""
+    import torch
+    _require_cuda(W)
+    if W.dtype != torch.float16:
+        raise TypeError("W must be float16")
+    K, N = W.shape
+    q8 = torch.empty((K, N), dtype=torch.int8, device=W.device)
+    S = torch.empty(((K + G - 1) // G, N), dtype=torch.float16, device=W.device)
+    _check(w8a16_quantize(W.contiguous(), q8, S, K, N, G, stream), "w8a16_quantize")
+    return q8, S
 
 
 def repack_w8(q, stream=None):

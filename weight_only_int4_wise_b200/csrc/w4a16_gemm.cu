@@ -896,7 +896,7 @@ void enumerate_tactics(int64_t M, int64_t N, int64_t K, int64_t G, bool need_dev
     *count = n;
 }
 
-constexpr int kMaxTactics = 64;
+constexpr int kMaxTactics = 96;
 
 int tactic_choice(int64_t M, int64_t N, int64_t K, int64_t G, int tactic, bool need_device, Choice* out) {
     Choice all[kMaxTactics];
@@ -1071,7 +1071,12 @@ std::atomic<long long> g_wait_limit{kTimeoutCycles};  // test aid: w4a16_set_fau
 std::atomic<int> g_stall_stage{-1};
 }
 
-bool static_weights_enabled() { return g_static_weights.load(std::memory_order_relaxed) != 0; }
+// Set by w4a16_gemm_ex for the duration of one call on this host thread.
+thread_local int t_call_static_weights = 0;
+
+bool static_weights_enabled() {
+    return t_call_static_weights != 0 || g_static_weights.load(std::memory_order_relaxed) != 0;
+}
 
 int sm_count() {
     static std::atomic<int> cached[64];
@@ -1469,4 +1474,15 @@ extern "C" int w8a16_gemm(const w4a16_half* A_dev, const uint8_t* Wt8_dev, const
     rc = plan_dense(M, N, K, &plan, true, 0, 0, 8);
     if (rc) return rc;
     return dense_launch(plan, 8, A_dev, Wt8_dev, S_dev, C_dev, M, N, K, G, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int w4a16_gemm_ex(const w4a16_half* A_dev, const uint8_t* Wt_dev, const w4a16_half* S_dev,
+                             w4a16_half* C_dev, int64_t M, int64_t N, int64_t K, int64_t G, uint32_t flags,
+                             void* stream) {
+    if (flags & ~static_cast<uint32_t>(W4A16_FLAG_STATIC_WEIGHTS)) return W4A16_ERR_INVALID_ARG;
+    struct CallScope {
+        explicit CallScope(int v) { t_call_static_weights = v; }
+        ~CallScope() { t_call_static_weights = 0; }
+    } scope((flags & W4A16_FLAG_STATIC_WEIGHTS) ? 1 : 0);
+    return w4a16_gemm(A_dev, Wt_dev, S_dev, C_dev, M, N, K, G, stream);
 }

@@ -48,47 +48,71 @@ constexpr int kSlices = 4;                  // row slices of a group in the stag
 constexpr int kMaxTmaGroup = 256;           // rows of one copy (the copy engine's box limit)
 constexpr long long kQuantTimeoutCycles = 4000000000ll;  // about 2 s at the boost clock
 
+// BITS = 4: int4 codes in [-8, 7], scale max/7, two codes per byte (row pairs).
+// BITS = 8: 8-bit codes in [-128, 127], scale max/127, one code per byte (the
+// W8A16 export step). The boundary window around a half-integer covers the
+// product's error (2 ulp of a quotient below 8, or below 128).
+template <int BITS>
+struct QuantRange {
+    static constexpr int kMin = BITS == 4 ? -8 : -128;
+    static constexpr int kMax = BITS == 4 ? 7 : 127;
+    static constexpr float kWindow = BITS == 4 ? 1e-5f : 1e-4f;
+};
+
 // Code of weight w with scale s (inverse rs = 1/s rounded): round(w / s), halves
-// away from zero, clamped to [-8, 7]; 0 when s = 0.
+// away from zero, clamped to the code range; 0 when s = 0.
+template <int BITS>
 __device__ __forceinline__ uint32_t quantize_code(float w, float s, float rs) {
     if (s == 0.0f) return 0u;
     float x = w * rs;
     const float a = fabsf(x);
-    if (fabsf(a - floorf(a) - 0.5f) < 1e-5f) x = __fdiv_rn(w, s);
+    if (fabsf(a - floorf(a) - 0.5f) < QuantRange<BITS>::kWindow) x = __fdiv_rn(w, s);
     int q = static_cast<int>(roundf(x));
-    q = q < -8 ? -8 : (q > 7 ? 7 : q);
-    return static_cast<uint32_t>(q) & 0xFu;
+    q = q < QuantRange<BITS>::kMin ? QuantRange<BITS>::kMin : (q > QuantRange<BITS>::kMax ? QuantRange<BITS>::kMax : q);
+    return static_cast<uint32_t>(q) & (BITS == 4 ? 0xFu : 0xFFu);
 }
 
+template <int BITS>
 __device__ __forceinline__ __half2 group_scales(float a0, float a1) {
-    return __halves2half2(__float2half_rn(__fdiv_rn(a0, 7.0f)), __float2half_rn(__fdiv_rn(a1, 7.0f)));
+    constexpr float kDiv = static_cast<float>(QuantRange<BITS>::kMax);
+    return __halves2half2(__float2half_rn(__fdiv_rn(a0, kDiv)), __float2half_rn(__fdiv_rn(a1, kDiv)));
 }
 
 // Rows 0..nrows-1 of one column pair, read through row(r), whose maxima are
-// (a0, a1): the pair's fp16 scales (stored at s_out), then one packed byte per
-// column and row pair, written from wp_row0 on with a stride of N2 16-bit words
-// per packed row.
-template <typename RowFn>
-__device__ __forceinline__ void quantize_pair(RowFn row, int64_t nrows, uint16_t* __restrict__ wp_row0,
+// (a0, a1): the pair's fp16 scales (stored at s_out), then the codes, written
+// from out_row0 on with a stride of N2 16-bit words per output row: for int4 one
+// packed byte per column and row pair (rows of the canonical packed layout), for
+// 8-bit codes one byte per column and row.
+template <int BITS, typename RowFn>
+__device__ __forceinline__ void quantize_pair(RowFn row, int64_t nrows, uint16_t* __restrict__ out_row0,
                                               int64_t N2, __half2* __restrict__ s_out, float a0, float a1) {
-    const __half2 sh = group_scales(a0, a1);
+    const __half2 sh = group_scales<BITS>(a0, a1);
     *s_out = sh;
     const float2 s = __half22float2(sh);
     const float r0 = s.x != 0.0f ? __frcp_rn(s.x) : 0.0f;
     const float r1 = s.y != 0.0f ? __frcp_rn(s.y) : 0.0f;
-    // Row pairs (k, k + 1): groups start on even rows (G is even), so a packed
-    // byte never spans two groups; a missing last odd row packs 0.
-    for (int64_t r = 0; r < nrows; r += 2) {
-        const float2 lo = __half22float2(row(r));
-        const bool two = r + 1 < nrows;
-        const float2 hi = two ? __half22float2(row(r + 1)) : make_float2(0.0f, 0.0f);
-        const uint32_t b0 = quantize_code(lo.x, s.x, r0) | (two ? quantize_code(hi.x, s.x, r0) << 4 : 0u);
-        const uint32_t b1 = quantize_code(lo.y, s.y, r1) | (two ? quantize_code(hi.y, s.y, r1) << 4 : 0u);
-        wp_row0[(r >> 1) * N2] = static_cast<uint16_t>(b0 | (b1 << 8));  // bytes of the pair's two columns
+    if constexpr (BITS == 4) {
+        // Row pairs (k, k + 1): groups start on even rows (G is even), so a packed
+        // byte never spans two groups; a missing last odd row packs 0.
+        for (int64_t r = 0; r < nrows; r += 2) {
+            const float2 lo = __half22float2(row(r));
+            const bool two = r + 1 < nrows;
+            const float2 hi = two ? __half22float2(row(r + 1)) : make_float2(0.0f, 0.0f);
+            const uint32_t b0 = quantize_code<4>(lo.x, s.x, r0) | (two ? quantize_code<4>(hi.x, s.x, r0) << 4 : 0u);
+            const uint32_t b1 = quantize_code<4>(lo.y, s.y, r1) | (two ? quantize_code<4>(hi.y, s.y, r1) << 4 : 0u);
+            out_row0[(r >> 1) * N2] = static_cast<uint16_t>(b0 | (b1 << 8));  // bytes of the pair's two columns
+        }
+    } else {
+        for (int64_t r = 0; r < nrows; ++r) {
+            const float2 v = __half22float2(row(r));
+            out_row0[r * N2] =
+                static_cast<uint16_t>(quantize_code<8>(v.x, s.x, r0) | (quantize_code<8>(v.y, s.y, r1) << 8));
+        }
     }
 }
 
 // Group g of a 256-column tile through shared memory (see the file header).
+template <int BITS>
 __global__ void __launch_bounds__(kQuantThreads * kSlices) quantize_tma_kernel(const __grid_constant__ CUtensorMap tmW,
                                                                       uint16_t* __restrict__ wp,
                                                                       __half2* __restrict__ S, int64_t K,
@@ -158,14 +182,16 @@ __global__ void __launch_bounds__(kQuantThreads * kSlices) quantize_tma_kernel(c
         }
         if (c < N2) {
             __half2 scratch;
-            quantize_pair([&](int64_t r) { return tile[(r0 + r) * kQuantThreads + t]; }, r1 - r0,
-                          wp + ((k0 + r0) >> 1) * N2 + c, N2, slice == 0 ? S + g * N2 + c : &scratch, a0, a1);
+            uint16_t* out = wp + (BITS == 4 ? ((k0 + r0) >> 1) : (k0 + r0)) * N2 + c;
+            quantize_pair<BITS>([&](int64_t r) { return tile[(r0 + r) * kQuantThreads + t]; }, r1 - r0, out, N2,
+                                slice == 0 ? S + g * N2 + c : &scratch, a0, a1);
         }
         __syncthreads();  // every thread is done with the tile and the partial maxima before they are reused
     }
 }
 
 // Fallback: the group's rows read twice from global memory (maximum, then codes).
+template <int BITS>
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __half2* __restrict__ W,
                                                                   uint16_t* __restrict__ wp,
                                                                   __half2* __restrict__ S, int64_t K,
@@ -182,8 +208,8 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __half2* 
             a0 = fmaxf(a0, fabsf(v.x));
             a1 = fmaxf(a1, fabsf(v.y));
         }
-        quantize_pair([&](int64_t r) { return W[(k0 + r) * N2 + c]; }, nrows, wp + (k0 >> 1) * N2 + c, N2,
-                      S + g * N2 + c, a0, a1);
+        quantize_pair<BITS>([&](int64_t r) { return W[(k0 + r) * N2 + c]; }, nrows,
+                            wp + (BITS == 4 ? (k0 >> 1) : k0) * N2 + c, N2, S + g * N2 + c, a0, a1);
     }
 }
 
@@ -193,12 +219,17 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __half2* 
 
 using namespace w4a16;
 
-extern "C" int w4a16_quantize(const w4a16_half* W_dev, uint8_t* wp_dev, w4a16_half* S_dev, int64_t K, int64_t N,
-                              int64_t G, void* stream) {
-    if (!W_dev || !wp_dev || !S_dev || K <= 0 || N <= 0 || G <= 0) return W4A16_ERR_INVALID_ARG;
+namespace {
+
+// Codes to out_dev (int4: canonical packed [ceil(K/2), N]; 8-bit: [K, N] int8),
+// scales to S_dev [ceil(K/G), N].
+template <int BITS>
+int quantize_launch(const w4a16_half* W_dev, void* out_dev, w4a16_half* S_dev, int64_t K, int64_t N, int64_t G,
+                    void* stream) {
+    if (!W_dev || !out_dev || !S_dev || K <= 0 || N <= 0 || G <= 0) return W4A16_ERR_INVALID_ARG;
     if ((N & 1) || (G & 1) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(W_dev) & 3u) || (reinterpret_cast<uintptr_t>(S_dev) & 3u) ||
-        (reinterpret_cast<uintptr_t>(wp_dev) & 1u))
+        (reinterpret_cast<uintptr_t>(out_dev) & 1u))
         return W4A16_ERR_MISALIGNED;
     int rc = check_device();
     if (rc) return rc;
@@ -217,21 +248,33 @@ extern "C" int w4a16_quantize(const w4a16_half* W_dev, uint8_t* wp_dev, w4a16_ha
         if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return W4A16_ERR_CUDA;
         const size_t smem = 128 + kSlices * kQuantThreads * 8 + static_cast<size_t>(kMaxTmaGroup) * kTileCols * 2;
         if (!attr_done[dev]) {
-            if (cudaFuncSetAttribute(reinterpret_cast<const void*>(quantize_tma_kernel),
+            if (cudaFuncSetAttribute(reinterpret_cast<const void*>(quantize_tma_kernel<BITS>),
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
                 cudaSuccess)
                 return W4A16_ERR_CUDA;
             attr_done[dev] = true;
         }
-        quantize_tma_kernel<<<grid, kQuantThreads * kSlices,
-                              128 + kSlices * kQuantThreads * 8 + static_cast<size_t>(G) * kTileCols * 2, st>>>(
-            map, reinterpret_cast<uint16_t*>(wp_dev), reinterpret_cast<__half2*>(S_dev), K, N, G, groups);
+        quantize_tma_kernel<BITS><<<grid, kQuantThreads * kSlices,
+                                    128 + kSlices * kQuantThreads * 8 + static_cast<size_t>(G) * kTileCols * 2, st>>>(
+            map, reinterpret_cast<uint16_t*>(out_dev), reinterpret_cast<__half2*>(S_dev), K, N, G, groups);
     } else {
-        quantize_kernel<<<grid, kQuantThreads, 0, st>>>(reinterpret_cast<const __half2*>(W_dev),
-                                                        reinterpret_cast<uint16_t*>(wp_dev),
-                                                        reinterpret_cast<__half2*>(S_dev), K, N, G, groups);
+        quantize_kernel<BITS><<<grid, kQuantThreads, 0, st>>>(reinterpret_cast<const __half2*>(W_dev),
+                                                              reinterpret_cast<uint16_t*>(out_dev),
+                                                              reinterpret_cast<__half2*>(S_dev), K, N, G, groups);
     }
     return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int w4a16_quantize(const w4a16_half* W_dev, uint8_t* wp_dev, w4a16_half* S_dev, int64_t K, int64_t N,
+                              int64_t G, void* stream) {
+    return quantize_launch<4>(W_dev, wp_dev, S_dev, K, N, G, stream);
+}
+
+extern "C" int w8a16_quantize(const w4a16_half* W_dev, int8_t* q8_dev, w4a16_half* S_dev, int64_t K, int64_t N,
+                              int64_t G, void* stream) {
+    return quantize_launch<8>(W_dev, q8_dev, S_dev, K, N, G, stream);
 }
 
 namespace w4a16 {
