@@ -183,7 +183,7 @@ def replay_stats(graph, launches_per_replay, reps):
             "mean": round(sum(samples) / len(samples), 3), "reps": reps, "launches_per_rep": launches_per_replay}
 
 
-SKINNY_SOURCES = ("w4a16_skinny.cu", "dequant.cuh", "ptx.cuh")
+SKINNY_SOURCES = ("w4a16_skinny.cu", "dequant.cuh", "epilogue.cuh", "ptx.cuh")
 
 
 def skinny_source_digest() -> str:
@@ -496,8 +496,9 @@ def run_ours(args):
                      "per direction with double batch buffers overlapping the neighbouring batches' GEMMs; two "
                      "w4a16_gemm calls per step"}
 
-    extra = per_config(w4, dev, tune=not args.no_tune) if (rank == 0 and not args.no_configs) else None
-    tactics = tactic_report(w4, dev) if (rank == 0 and not args.no_configs) else None
+    only = [x for x in args.configs.split(",") if x] if args.configs else None
+    extra = per_config(w4, dev, tune=not args.no_tune, only=only) if (rank == 0 and not args.no_configs) else None
+    tactics = tactic_report(w4, dev) if (rank == 0 and not args.no_configs and not only) else None
     peaks = load_peaks()
     achieved = K * step_bytes() / sec / 1e9  # per GPU: every launch in the step is the same kernel
     line = {
@@ -600,7 +601,7 @@ def tactic_report(w4, dev):
     return out
 
 
-def per_config(w4, dev, tune=True):
+def per_config(w4, dev, tune=True, only=None):
     """Device time per launch for every workload family (context for the headline line).
     Dense W4A16 shapes run the autotuned launch form (unless tune is False)."""
     import torch
@@ -608,7 +609,7 @@ def per_config(w4, dev, tune=True):
     l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20)
     out = {}
     for name, cfg in workloads.CONFIGS.items():
-        if name == "tiny":
+        if name == "tiny" or (only and name not in only):
             continue
         c = workloads.make(name)
         tactic = None
@@ -677,9 +678,15 @@ def per_config(w4, dev, tune=True):
                     raise RuntimeError(w4.status_string(rc))
             rows = c.tokens * c.top_k
             fl = 2 * flops(rows, c.I, c.H)
-            # both projections' weights and scales, activations in and out of each, the
-            # gather and the combine; every expert receives rows at this size
-            by = c.E * (algorithmic_bytes(0, c.I, c.H, c.G) + algorithmic_bytes(0, c.H, c.I, c.G)) + \
+            # experts that receive rows (the GPU's own routing of these logits)
+            ids = torch.empty((c.tokens, c.top_k), dtype=torch.int32, device=dev)
+            wts_r = torch.empty((c.tokens, c.top_k), dtype=torch.float32, device=dev)
+            if w4.w4a16_moe_route(lg, ids, wts_r, c.tokens, c.E, c.top_k):
+                raise RuntimeError("routing failed")
+            active = int(torch.unique(ids).numel())
+            # the active experts' weights and scales of both projections, activations in
+            # and out of each, the gather and the combine
+            by = active * (algorithmic_bytes(0, c.I, c.H, c.G) + algorithmic_bytes(0, c.H, c.I, c.G)) + \
                 rows * (c.H + c.I) * 2 * 2 + (c.tokens * c.H * 2) * 2 + rows * c.H * 2 * 2
         else:
             wts = [w4.prepare_weights(torch.from_numpy(c.q[e]).to(dev))[1] for e in range(c.E)]
@@ -721,9 +728,12 @@ def per_config(w4, dev, tune=True):
                                                                   f"{n} launches each"}
         if tactic is not None:
             out[name]["tactic"] = tactic
+        if cfg["kind"] == "moe":
+            out[name]["active_experts"] = active
         del g
-    out["quantize"] = quantize_timing(w4, dev, peaks, l2)
-    out["quantize_w8"] = quantize_timing(w4, dev, peaks, l2, bits=8)
+    if not only or "quantize" in only:
+        out["quantize"] = quantize_timing(w4, dev, peaks, l2)
+        out["quantize_w8"] = quantize_timing(w4, dev, peaks, l2, bits=8)
     status = w4.device_status(clear=True)
     if status != w4.OK:
         raise RuntimeError(f"device status after per-config timing: {w4.status_string(status)}")
@@ -874,6 +884,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config timings")
+    ap.add_argument("--configs", default="", help="comma-separated subset of the per-config timings")
     ap.add_argument("--no-tune", action="store_true",
                     help="per-config timings with the built-in heuristic instead of autotuned launch forms")
     ap.add_argument("--tune-headline", action="store_true",

@@ -164,6 +164,28 @@ def test_up_projection_with_activation(o, act):
         assert d.max() <= 1 and np.count_nonzero(d) <= max(4, d.size // 1000)
 
 
+@pytest.mark.parametrize("act", ACTS)
+def test_up_projection_activation_on_the_skinny_kernel(o, act):
+    # 12 gathered rows: the grouped product with its activation runs on the skinny kernel
+    c = workloads.grouped(E=4, top_k=2, tokens=6, K=1024, N=264, G=128, seed=95 + act)
+    wts = [device_weights(c.q[e])[1] for e in range(c.E)]
+    Ss = [dev(c.S[e]) for e in range(c.E)]
+    A, off = dev(c.A), dev(c.offsets)
+    assert w.w4a16_grouped_launch_info(c.E, c.total_rows, c.N, c.K, c.G)[1].token_tile == 16
+    h = torch.empty((c.total_rows, c.N), dtype=torch.float16, device="cuda")
+    a = torch.empty_like(h)
+    assert w.w4a16_grouped_gemm_act(A, wts, Ss, off, h, c.E, c.total_rows, c.N, c.K, c.G, moe.ACT_IDENTITY) == w.OK
+    assert w.w4a16_grouped_gemm_act(A, wts, Ss, off, a, c.E, c.total_rows, c.N, c.K, c.G, act) == w.OK
+    torch.cuda.synchronize()
+    h, a = h.cpu().numpy(), a.cpu().numpy()
+    ref_h = o.grouped_gemm(c.A, [pins.python_pack(c.q[e]) for e in range(c.E)], list(c.S), c.offsets, c.K, c.G)
+    ok, err, _ = within_tolerance(h, ref_h)
+    assert ok, err
+    d = ulp_diff(a, moe.activation(h, act))
+    assert d.max() <= (0 if act in (moe.ACT_IDENTITY, moe.ACT_RELU) else 1)
+    assert w.device_status() == w.OK
+
+
 def test_combine_within_one_ulp():
     T, k, H = 333, 2, 512
     g = np.random.Generator(np.random.PCG64(8))

@@ -211,6 +211,22 @@ def test_grouped_rejects_malformed_offsets_on_device():
         assert guards_intact(flat, pad, 0) and np.all(C.cpu().numpy().view(np.uint16) == 0x7BAD)
 
 
+@pytest.mark.parametrize("tokens,E,k,K,N,G", [
+    (1, 8, 1, 512, 256, 128),    # one row: seven experts without rows
+    (4, 8, 2, 1024, 392, 128),   # 8 rows, one token tile, ragged column tile
+    (8, 6, 2, 1024, 264, 48),    # 16 rows, two token tiles, groups straddling blocks
+    (3, 4, 3, 4096, 512, 64),    # 9 rows, a K split over a cluster
+    (16, 8, 1, 256, 128, 32),
+])
+def test_grouped_decode_batches_run_on_the_skinny_kernel(o, tokens, E, k, K, N, G):
+    # at most 16 gathered rows in all: the grouped product runs on the skinny kernel, one
+    # grid slice per expert, experts without rows skipped
+    c = workloads.grouped(E=E, top_k=k, tokens=tokens, K=K, N=N, G=G, seed=tokens * 11 + K)
+    rc, info = w.w4a16_grouped_launch_info(c.E, c.total_rows, c.N, c.K, c.G)
+    assert rc == w.OK and info.token_tile in (8, 16) and info.grid_z == E
+    run_grouped(o, c)
+
+
 def test_misaligned_pointer_is_refused():
     c = workloads.dense(4, 128, 128, 64, 35)
     _, wt = device_weights(c.q)

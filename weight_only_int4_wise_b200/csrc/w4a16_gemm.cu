@@ -48,6 +48,7 @@
 
 #include "../../include/w4a16.h"
 #include "dequant.cuh"
+#include "epilogue.cuh"
 #include "ptx.cuh"
 #include "w4a16_internal.h"
 
@@ -113,28 +114,6 @@ struct Layout {
 
 __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
 
-// Epilogue value: the fp32 accumulator rounded to fp16 (the product's result),
-// then, for the expert layer's up projection, the activation evaluated in fp32
-// on that fp16 value and rounded to fp16 again. GELU in both of its usual
-// forms: x * Phi(x) with Phi the normal CDF (erf form), and the tanh
-// approximation with the cubic term 0.044715 x^3. Both are written without
-// the sum 1 + (something near -1) that loses all of fp32's digits for negative
-// x: Phi(x) = erfc(-x / sqrt 2) / 2, and (1 + tanh u) / 2 = 1 / (1 + e^(-2u)).
-__device__ __forceinline__ __half epilogue_value(float acc, int act) {
-    const __half h = __float2half_rn(acc);
-    if (act == W4A16_ACT_IDENTITY) return h;
-    const float x = __half2float(h);
-    float y;
-    if (act == W4A16_ACT_RELU) {
-        y = fmaxf(x, 0.f);
-    } else if (act == W4A16_ACT_GELU_ERF) {
-        y = 0.5f * x * erfcf(x * -0.70710678118654752f);
-    } else {
-        const float u = 0.79788456080286536f * (x + 0.044715f * x * x * x);
-        y = x / (1.f + expf(-2.f * u));
-    }
-    return __float2half_rn(y);
-}
 
 // Bounded wait on an mbarrier phase. Returns false if the CTA is aborting or
 // the wait ran out (which starts the abort). The bound is counted in SM clock
@@ -1136,6 +1115,12 @@ extern "C" int w4a16_grouped_launch_info(int64_t E, int64_t total_rows, int64_t 
     if (rc) return rc;
     if (total_rows >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
     const bool dev = check_device() == W4A16_OK;
+    SkinnyPlan sk;
+    if (skinny_plan_grouped(total_rows, N, K, G, &sk) == W4A16_OK) {
+        fill_info_skinny(sk, info);
+        info->grid_z = static_cast<int32_t>(E);
+        return W4A16_OK;
+    }
     Plan plan;
     rc = plan_grouped(E, total_rows, N, K, &plan, dev);
     if (rc) return rc;
@@ -1224,6 +1209,10 @@ int grouped_gemm_act(const w4a16_half* A_dev, const uint8_t* const* Wt, const w4
     if (total_rows == 0) return W4A16_OK;
     rc = check_device();
     if (rc) return rc;
+    SkinnyPlan sk;
+    if (skinny_plan_grouped(total_rows, N, K, G, &sk) == W4A16_OK)  // decode-sized batches: at most 16 rows in all
+        return skinny_grouped_launch(sk, A_dev, Wt, reinterpret_cast<const void* const*>(S), offsets_dev, C_dev, E,
+                                     total_rows, N, K, G, act, stream);
     Plan plan;
     rc = plan_grouped(E, total_rows, N, K, &plan, true);
     if (rc) return rc;

@@ -75,4 +75,18 @@ int skinny_device_status(bool clear);
 int skinny_launch(const SkinnyPlan& plan, const void* A, const uint8_t* Wt, const void* S, void* C, int64_t M,
                   int64_t N, int64_t K, int64_t G, cudaStream_t stream);
 
+// The skinny plan of the grouped form: the smallest K split whose staged
+// activations fit (the experts' column tiles already fill the grid).
+int skinny_plan_grouped(int64_t total_rows, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan);
+
+// Grouped-expert form of the skinny kernel (grid z = expert) for at most 16
+// gathered rows in total (plan from skinny_plan_grouped): rows
+// [off[e], off[e+1]) of A and C use Wt[e] and S[e] (host arrays of E device
+// pointers); the activation act (W4A16_ACT_*) applies to the fp16 result.
+// Malformed offsets (or a segment longer than the plan's token tiles) latch
+// W4A16_ERR_BAD_OFFSETS in the skinny status word and write nothing.
+int skinny_grouped_launch(const SkinnyPlan& plan, const void* A, const uint8_t* const* Wt, const void* const* S,
+                          const int32_t* offsets, void* C, int64_t E, int64_t total_rows, int64_t N, int64_t K,
+                          int64_t G, int act, cudaStream_t stream);
+
 }  // namespace w4a16

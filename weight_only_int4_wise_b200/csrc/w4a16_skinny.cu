@@ -28,9 +28,11 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 
 #include "../../include/w4a16.h"
 #include "dequant.cuh"
+#include "epilogue.cuh"
 #include "ptx.cuh"
 #include "w4a16_internal.h"
 
@@ -44,8 +46,7 @@ constexpr int kBlockK = 128;
 constexpr int kSlotBytes = 32;                    // per thread and block: two 16-byte chunks
 
 // No wait in this kernel can fail to end (cp.async groups and cluster barriers
-// only), so its status word stays 0; it is kept so the device-status query has
-// one word per kernel family.
+// only); its status word latches malformed expert offsets in grouped mode.
 __device__ int g_skinny_status;
 
 struct SkinnyParams {
@@ -61,16 +62,50 @@ struct SkinnyParams {
     uint32_t g_magic;         // floor(k / G) == (k * g_magic) >> 32 for every k < K padded
     int32_t post_scale;       // G % 128 == 0: scale fp32 partials once per block
     int32_t prefetch;         // weights/scales may be read before the previous kernel finishes
+    // Grouped-expert mode (grid z = expert): rows [off[e], off[e+1]) of A and C
+    // use expert e's weights and scales; M is then the total row count.
+    int32_t grouped, E, act;  // act: W4A16_ACT_* applied to the fp16 result
+    const int32_t* offsets;
+    const uint8_t* wte[W4A16_MAX_EXPERTS];
+    const __half* sce[W4A16_MAX_EXPERTS];
 };
 
 // KH = 2 runs two sets of 8 warps over the same 128 columns, the first taking
 // the even 128-deep blocks of the CTA's K range and the second the odd ones, and
 // adds the two partial tiles in shared memory (first + second) after the loop.
-template <int MT, int kDepth, int KH>
+// GROUPED: the grouped-expert form (a separate instantiation, so that the
+// dense kernels keep their register budget).
+template <int MT, int kDepth, int KH, bool GROUPED>
 __global__ void __launch_bounds__(KH * kSkThreads, 2)
     w4a16_skinny_kernel(const __grid_constant__ SkinnyParams p) {
     extern __shared__ __align__(1024) uint8_t sm[];
     constexpr int kThreads = KH * kSkThreads;
+    // This CTA's operands: the whole product, or in grouped mode its expert's
+    // row segment (every CTA of a cluster has the same expert, so a cluster
+    // leaves together).
+    const uint8_t* Wt = p.wt;
+    const __half* Sc = p.sc;
+    const __half* Ap = p.A;
+    __half* Cp = p.C;
+    int Mrows = p.M;
+    if constexpr (GROUPED) {
+        grid_dependency_wait();  // the offsets come from the previous kernel
+        const int32_t* off = p.offsets;
+        bool ok = off[0] == 0 && off[p.E] == p.M;
+        for (int x = 0; x < p.E && ok; ++x) ok = off[x + 1] >= off[x] && off[x + 1] - off[x] <= 8 * MT;
+        if (!ok) {
+            if (threadIdx.x == 0) atomicCAS(&g_skinny_status, 0, W4A16_ERR_BAD_OFFSETS);
+            return;
+        }
+        const int e = blockIdx.z;
+        const int m0 = off[e];
+        Mrows = off[e + 1] - m0;
+        if (Mrows == 0) return;
+        Wt = p.wte[e];
+        Sc = p.sce[e];
+        Ap = p.A + static_cast<int64_t>(m0) * p.K;
+        Cp = p.C + static_cast<int64_t>(m0) * p.N;
+    }
     const int warp = (threadIdx.x >> 5) & (kSkWarps - 1), lane = threadIdx.x & 31;
     const int kh = static_cast<int>(threadIdx.x) / kSkThreads;  // K half: blocks i with i % KH == kh
     const int g = lane >> 2, t = lane & 3;
@@ -96,7 +131,7 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
 
     // This thread's chunk t of columns ja and ja + 8 in block i: tile 2(b0+i) + t/2,
     // half t%2. A missing second tile at an odd end of K reads as zeros.
-    const uint8_t* wsrc = p.wt + (static_cast<int64_t>(nt) * p.KT + 2 * b0 + (t >> 1)) * 4096 + (t & 1) * 2048 + ja * 16;
+    const uint8_t* wsrc = Wt + (static_cast<int64_t>(nt) * p.KT + 2 * b0 + (t >> 1)) * 4096 + (t & 1) * 2048 + ja * 16;
     const int kt_last_ok = p.KT - 1 - (t >> 1);
     uint8_t* myslot = ring + threadIdx.x * 16;  // chunk of column ja; column ja + 8's is kThreads * 16 further
     // Local block li of this half is block i = li * KH + kh, in slot li % kDepth.
@@ -106,8 +141,8 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
             const bool ok = 2 * (b0 + i) <= kt_last_ok;
             const uint8_t* src = wsrc + static_cast<int64_t>(i) * 8192;
             uint8_t* dst = myslot + (li % kDepth) * kThreads * kSlotBytes;
-            cp_async16(dst, ok ? src : p.wt, ok ? 16u : 0u);
-            cp_async16(dst + kThreads * 16, ok ? src + 128 : p.wt, ok ? 16u : 0u);
+            cp_async16(dst, ok ? src : Wt, ok ? 16u : 0u);
+            cp_async16(dst + kThreads * 16, ok ? src + 128 : Wt, ok ? 16u : 0u);
         }
         cp_async_commit();  // one group per block, empty past the end, so the counts stay uniform
     };
@@ -117,7 +152,7 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
             const int r = idx >> 4, c = idx & 15;
             const bool ok = c * 8 < ncols;
             cp_async16(scl + r * 128 + c * 8,
-                       ok ? p.sc + static_cast<int64_t>(g_lo + r) * p.N + nt * 128 + c * 8 : p.sc, ok ? 16u : 0u);
+                       ok ? Sc + static_cast<int64_t>(g_lo + r) * p.N + nt * 128 + c * 8 : Sc, ok ? 16u : 0u);
         }
         cp_async_commit();  // the oldest group: complete by the time block 0 is
     };
@@ -145,7 +180,7 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
             const int r = idx / cpr, c = idx - r * cpr;
             const int k = kr0 + c * 8;
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (r < p.M && k < p.K) v = *reinterpret_cast<const uint4*>(p.A + static_cast<int64_t>(r) * p.K + k);
+            if (r < Mrows && k < p.K) v = *reinterpret_cast<const uint4*>(Ap + static_cast<int64_t>(r) * p.K + k);
             *reinterpret_cast<uint4*>(act + r * p.act_stride + c * 8) = v;
         }
     }
@@ -271,7 +306,9 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
             for (int e = 0; e < 4; ++e) {
                 const int m = m0 + (e & 1);
                 const int n = na + ((e >> 1) << 3);
-                if (m < p.M && n < p.N) p.C[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(acc[j][e]);
+                if (m < Mrows && n < p.N)
+                    Cp[static_cast<int64_t>(m) * p.N + n] =
+                        GROUPED ? epilogue_value(acc[j][e], p.act) : __float2half_rn(acc[j][e]);
             }
         }
         return;
@@ -293,20 +330,20 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
                 const int col = ja + ((e >> 1) << 3);
                 const int q = (col * S) >> 7;          // owner of this column
                 const int cq = (q * 128 + S - 1) / S;  // owner's first column
-                if (m < p.M)
+                if (m < Mrows)
                     st_dsmem_f32(&red[(rank * MP + m) * cwm + (col - cq)], static_cast<uint32_t>(q), acc[j][e]);
             }
         }
     }
     cluster_sync_all();
     const int c0 = (rank * 128 + S - 1) / S, c1 = ((rank + 1) * 128 + S - 1) / S, cw = c1 - c0;
-    for (int o = threadIdx.x; o < cw * p.M; o += kThreads) {
+    for (int o = threadIdx.x; o < cw * Mrows; o += kThreads) {
         const int m = o / cw, c = o - m * cw;
         const int n = nt * 128 + c0 + c;
         if (n < p.N) {
             float sum = 0.f;
             for (int r = 0; r < S; ++r) sum += red[(r * MP + m) * cwm + c];
-            p.C[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(sum);
+            Cp[static_cast<int64_t>(m) * p.N + n] = GROUPED ? epilogue_value(sum, p.act) : __float2half_rn(sum);
         }
     }
 }
@@ -399,6 +436,23 @@ int skinny_plan(int64_t M, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan) {
     }
 }
 
+int skinny_plan_grouped(int64_t total_rows, int64_t N, int64_t K, int64_t G, SkinnyPlan* plan) {
+    // The experts' column tiles already give E x ceil(N/128) CTAs, so K is split
+    // only as far as the staged activations need to fit in shared memory.
+    if (total_rows < 1 || total_rows > kSkinnyMaxM) return W4A16_ERR_UNSUPPORTED;
+    const int64_t KB = ((K + 63) / 64 + 1) / 2;
+    const int mt = total_rows <= 8 ? 1 : 2;
+    for (int64_t splits = 1; splits <= 8 && splits <= KB; ++splits) {
+        const int64_t nbmax = (KB + splits - 1) / splits;
+        const int kh = k_halves(mt, nbmax);
+        const int64_t nbh = (nbmax + kh - 1) / kh;
+        const int deep = nbh <= (8 / kh) / 2 ? 0 : 1;
+        if (skinny_plan_fill(total_rows, N, K, G, static_cast<int>(splits), kh, deep, plan) == W4A16_OK)
+            return W4A16_OK;
+    }
+    return W4A16_ERR_UNSUPPORTED;
+}
+
 int skinny_device_status(bool clear) {
     int v = 0;
     if (cudaMemcpyFromSymbol(&v, g_skinny_status, sizeof(int)) != cudaSuccess) return -1;
@@ -409,17 +463,24 @@ int skinny_device_status(bool clear) {
     return v;
 }
 
-int skinny_launch(const SkinnyPlan& plan, const void* A, const uint8_t* Wt, const void* S, void* C, int64_t M,
-                  int64_t N, int64_t K, int64_t G, cudaStream_t stream) {
-    static bool attr_done[6][64] = {};
+namespace {
+
+// Launch with filled parameters; grid z = 1 (dense) or the number of experts.
+int skinny_launch_params(const SkinnyPlan& plan, SkinnyParams& p, int64_t N, int64_t K, int64_t G, unsigned grid_z,
+                         cudaStream_t stream) {
+    static bool attr_done[12][64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return W4A16_ERR_CUDA;
     const int kh = plan.threads / kSkThreads;
-    const int vi = (plan.mt == 2 ? 4 : (kh == 2 ? 2 : 0)) + (plan.depth == 8 / kh ? 1 : 0);
+    const int vi = (p.grouped ? 6 : 0) + (plan.mt == 2 ? 4 : (kh == 2 ? 2 : 0)) + (plan.depth == 8 / kh ? 1 : 0);
     // (shared-memory carve-out: the largest, so two CTAs fit per SM)
-    void (*kernels[6])(SkinnyParams) = {w4a16_skinny_kernel<1, 4, 1>, w4a16_skinny_kernel<1, 8, 1>,
-                                        w4a16_skinny_kernel<1, 2, 2>, w4a16_skinny_kernel<1, 4, 2>,
-                                        w4a16_skinny_kernel<2, 4, 1>, w4a16_skinny_kernel<2, 8, 1>};
+    void (*kernels[12])(SkinnyParams) = {
+        w4a16_skinny_kernel<1, 4, 1, false>, w4a16_skinny_kernel<1, 8, 1, false>,
+        w4a16_skinny_kernel<1, 2, 2, false>, w4a16_skinny_kernel<1, 4, 2, false>,
+        w4a16_skinny_kernel<2, 4, 1, false>, w4a16_skinny_kernel<2, 8, 1, false>,
+        w4a16_skinny_kernel<1, 4, 1, true>,  w4a16_skinny_kernel<1, 8, 1, true>,
+        w4a16_skinny_kernel<1, 2, 2, true>,  w4a16_skinny_kernel<1, 4, 2, true>,
+        w4a16_skinny_kernel<2, 4, 1, true>,  w4a16_skinny_kernel<2, 8, 1, true>};
     if (!attr_done[vi][dev]) {
         if (cudaFuncSetAttribute(reinterpret_cast<const void*>(kernels[vi]),
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess ||
@@ -429,12 +490,6 @@ int skinny_launch(const SkinnyPlan& plan, const void* A, const uint8_t* Wt, cons
             return W4A16_ERR_CUDA;
         attr_done[vi][dev] = true;
     }
-    SkinnyParams p;
-    p.wt = Wt;
-    p.sc = reinterpret_cast<const __half*>(S);
-    p.A = reinterpret_cast<const __half*>(A);
-    p.C = reinterpret_cast<__half*>(C);
-    p.M = static_cast<int32_t>(M);
     p.N = static_cast<int32_t>(N);
     p.K = static_cast<int32_t>(K);
     p.G = static_cast<int32_t>(G);
@@ -446,10 +501,9 @@ int skinny_launch(const SkinnyPlan& plan, const void* A, const uint8_t* Wt, cons
     p.scale_rows = plan.scale_rows;
     p.g_magic = plan.g_magic;
     p.post_scale = plan.post_scale;
-    p.prefetch = static_weights_enabled() ? 1 : 0;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(plan.grid_x), static_cast<unsigned>(plan.grid_y), 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(plan.grid_x), static_cast<unsigned>(plan.grid_y), grid_z);
     cfg.blockDim = dim3(static_cast<unsigned>(plan.threads), 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem);
     cfg.stream = stream;
@@ -469,6 +523,43 @@ int skinny_launch(const SkinnyPlan& plan, const void* A, const uint8_t* Wt, cons
     cfg.numAttrs = na;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernels[vi], p);
     return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+}  // namespace
+
+int skinny_launch(const SkinnyPlan& plan, const void* A, const uint8_t* Wt, const void* S, void* C, int64_t M,
+                  int64_t N, int64_t K, int64_t G, cudaStream_t stream) {
+    SkinnyParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.wt = Wt;
+    p.sc = reinterpret_cast<const __half*>(S);
+    p.A = reinterpret_cast<const __half*>(A);
+    p.C = reinterpret_cast<__half*>(C);
+    p.M = static_cast<int32_t>(M);
+    p.prefetch = static_weights_enabled() ? 1 : 0;
+    return skinny_launch_params(plan, p, N, K, G, 1, stream);
+}
+
+int skinny_grouped_launch(const SkinnyPlan& plan, const void* A, const uint8_t* const* Wt, const void* const* S,
+                          const int32_t* offsets, void* C, int64_t E, int64_t total_rows, int64_t N, int64_t K,
+                          int64_t G, int act, cudaStream_t stream) {
+    SkinnyParams p;
+    std::memset(&p, 0, sizeof(p));
+    for (int64_t e = 0; e < E; ++e) {
+        p.wte[e] = Wt[e];
+        p.sce[e] = reinterpret_cast<const __half*>(S[e]);
+    }
+    p.wt = Wt[0];
+    p.sc = reinterpret_cast<const __half*>(S[0]);
+    p.A = reinterpret_cast<const __half*>(A);
+    p.C = reinterpret_cast<__half*>(C);
+    p.M = static_cast<int32_t>(total_rows);
+    p.grouped = 1;
+    p.E = static_cast<int32_t>(E);
+    p.act = act;
+    p.offsets = offsets;
+    p.prefetch = 0;  // the expert of a CTA is known only after the offsets, which follow the wait
+    return skinny_launch_params(plan, p, N, K, G, static_cast<unsigned>(E), stream);
 }
 
 }  // namespace w4a16

@@ -162,6 +162,8 @@ CONFIGS: Dict[str, dict] = {
     # the whole mixture-of-experts layer around the grouped product (up 4096 -> 14336,
     # down 14336 -> 4096), routed by its own logits
     "moe_layer":   dict(kind="moe", E=8, top_k=2, tokens=512, H=4096, I=14336, G=128, seed=6),
+    # the same layer at a decode batch of 4 tokens (8 gathered rows)
+    "moe_decode":  dict(kind="moe", E=8, top_k=2, tokens=4, H=4096, I=14336, G=128, seed=9),
     # the 8-bit code variant (W8A16) at the decode and prefill sizes
     "w8_decode_m16": dict(kind="dense8", M=16, K=4096, N=4096, G=128, seed=7),
     "w8_prefill":    dict(kind="dense8", M=2048, K=4096, N=4096, G=128, seed=8),
