@@ -57,7 +57,7 @@ struct SkinnyParams {
     int32_t M, N, K, G;
     int32_t ngroups, KT, KB;  // groups, 64-deep tiles, 128-deep blocks
     int32_t splits;
-    int32_t act_stride;       // halves per staged activation row (max K range + 8)
+    int32_t act_stride;       // halves per staged activation row (max K range + 16)
     int32_t scale_rows;       // rows of the staged scale window
     uint32_t g_magic;         // floor(k / G) == (k * g_magic) >> 32 for every k < K padded
     int32_t post_scale;       // G % 128 == 0: scale fp32 partials once per block
@@ -181,7 +181,14 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
             const int k = kr0 + c * 8;
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
             if (r < Mrows && k < p.K) v = *reinterpret_cast<const uint4*>(Ap + static_cast<int64_t>(r) * p.K + k);
-            *reinterpret_cast<uint4*>(act + r * p.act_stride + c * 8) = v;
+            // Within each 128-deep block the 4-wide k groups are interleaved: group
+            // (t, s) (k = 32t + 4s .. +3, thread column t's step s) sits at halves
+            // 16s + 4t. With rows 16 halves (32 bytes mod 128) apart, the 32 lanes'
+            // 8-byte fragment loads of one step then hit distinct banks.
+            const int q = c & 3, t4 = (c >> 2) & 3;
+            __half* rowp = act + r * p.act_stride + (c >> 4) * 128 + 32 * q + 4 * t4;
+            *reinterpret_cast<uint2*>(rowp) = make_uint2(v.x, v.y);
+            *reinterpret_cast<uint2*>(rowp + 16) = make_uint2(v.z, v.w);
         }
     }
     cp_async_wait<kDepth - 1>();  // the scale rows (and this thread's first block) have landed
@@ -198,7 +205,7 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
     }
     uint32_t arow[MT];
 #pragma unroll
-    for (int j = 0; j < MT; ++j) arow[j] = smem_addr(act + (8 * j + g) * p.act_stride + 32 * t);
+    for (int j = 0; j < MT; ++j) arow[j] = smem_addr(act + (8 * j + g) * p.act_stride + 4 * t);
     const uint32_t slot0 = smem_addr(myslot);
 
     const int nbh = (nb - kh + KH - 1) / KH;  // blocks of this half
@@ -227,7 +234,7 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
                     const int st = 2 * w + u;
 #pragma unroll
                     for (int j = 0; j < MT; ++j) {
-                        const uint2 bfr = lds64(arow[j] + kb2 + 8 * st);
+                        const uint2 bfr = lds64(arow[j] + kb2 + 32 * st);
                         if (w == 0)
                             mma_m16n8k16_zc(part[u][j], afr, bfr.x, bfr.y);
                         else
@@ -260,7 +267,7 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
                     const int st = 2 * w + u;
 #pragma unroll
                     for (int j = 0; j < MT; ++j) {
-                        const uint2 bfr = lds64(arow[j] + kb2 + 8 * st);
+                        const uint2 bfr = lds64(arow[j] + kb2 + 32 * st);
                         mma_m16n8k16(u ? acc2[j] : acc[j], afr, bfr.x, bfr.y);  // two chains
                     }
                 }
@@ -374,7 +381,7 @@ int skinny_plan_fill(int64_t M, int64_t N, int64_t K, int64_t G, int splits, int
     const int dmax = 8 / kh;  // 128-deep blocks in flight per thread: 8 per CTA
     const int depth = deep ? dmax : dmax / 2;
     const int64_t krange = nbmax * kBlockK;
-    const int64_t stride = krange + 8;
+    const int64_t stride = krange + 16;  // 32 bytes mod 128 between rows (see the staging loop)
     const int64_t rows = krange / G + 2;
     const int64_t bytes =
         smem_bytes(kh, depth, mt, splits, static_cast<int>(stride), static_cast<int>(rows));
