@@ -296,11 +296,15 @@ def run_ours(args):
     S0 = torch.from_numpy(case.S).to(dev)
     A0 = torch.from_numpy(case.A).to(dev)
     l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20)
-    copy_bytes = wt0.numel() + S0.numel() * 2 + A0.numel() * 2
+    # Weights and scales rotate over copies that together exceed L2 twice, so every
+    # launch streams its weights from HBM. The activations come from one buffer,
+    # as a decoder layer's input comes from the kernel before it (still in L2);
+    # --cold-activations rotates them with the weights instead.
+    copy_bytes = wt0.numel() + S0.numel() * 2 + (A0.numel() * 2 if args.cold_activations else 0)
     R = max(3, math.ceil(2 * l2 / copy_bytes) + 1)
     wts = [wt0] + [wt0.clone() for _ in range(R - 1)]
     Ss = [S0] + [S0.clone() for _ in range(R - 1)]
-    As = [A0] + [A0.clone() for _ in range(R - 1)]
+    As = [A0] + [A0.clone() if args.cold_activations else A0 for _ in range(R - 1)]
     C1 = torch.empty((1, N_DIM), dtype=torch.float16, device=dev)
     C16 = torch.empty((16, N_DIM), dtype=torch.float16, device=dev)
     outs = {1: C1, 16: C16}
@@ -506,8 +510,12 @@ def run_ours(args):
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "M": list(M_STEP), "K": K_DIM, "N": N_DIM, "G": G_DIM,
-                   "l2": f"inputs larger than L2: {R} rotating copies of weights+scales+activations "
-                         f"({R * copy_bytes / 2 ** 20:.0f} MiB vs {l2 / 2 ** 20:.0f} MiB L2)",
+                   "l2": (f"inputs larger than L2: {R} rotating copies of weights+scales+activations "
+                          f"({R * copy_bytes / 2 ** 20:.0f} MiB vs {l2 / 2 ** 20:.0f} MiB L2)"
+                          if args.cold_activations else
+                          f"inputs larger than L2: {R} rotating copies of weights+scales "
+                          f"({R * copy_bytes / 2 ** 20:.0f} MiB vs {l2 / 2 ** 20:.0f} MiB L2); the activations "
+                          f"come from one buffer, as a layer's input comes from the kernel before it"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "static_weights": True,
                    "launch": "CUDA graphs, programmatic dependent launch" +
@@ -618,9 +626,10 @@ def per_config(w4, dev, tune=True, only=None):
             S = torch.from_numpy(c.S).to(dev)
             A = torch.from_numpy(c.A).to(dev)
             C = torch.empty((c.M, c.N), dtype=torch.float16, device=dev)
-            per = wt.numel() + S.numel() * 2 + A.numel() * 2 + C.numel() * 2
+            # weights and scales rotate (from HBM); activations and output stay in one buffer
+            per = wt.numel() + S.numel() * 2
             R = max(2, math.ceil(2 * l2 / per) + 1)
-            bufs = [(wt, S, A, C)] + [(wt.clone(), S.clone(), A.clone(), torch.empty_like(C)) for _ in range(R - 1)]
+            bufs = [(wt, S, A, C)] + [(wt.clone(), S.clone(), A, C) for _ in range(R - 1)]
             M, N, K, G = c.M, c.N, c.K, c.G
 
             def launch(r, b=bufs, M=M, N=N, K=K, G=G):
@@ -641,9 +650,10 @@ def per_config(w4, dev, tune=True, only=None):
             S = torch.from_numpy(c.S).to(dev)
             A = torch.from_numpy(c.A).to(dev)
             C = torch.empty((c.M, c.N), dtype=torch.float16, device=dev)
-            per = wt.numel() + S.numel() * 2 + A.numel() * 2 + C.numel() * 2
+            # weights and scales rotate (from HBM); activations and output stay in one buffer
+            per = wt.numel() + S.numel() * 2
             R = max(2, math.ceil(2 * l2 / per) + 1)
-            bufs = [(wt, S, A, C)] + [(wt.clone(), S.clone(), A.clone(), torch.empty_like(C)) for _ in range(R - 1)]
+            bufs = [(wt, S, A, C)] + [(wt.clone(), S.clone(), A, C) for _ in range(R - 1)]
             M, N, K, G = c.M, c.N, c.K, c.G
 
             def launch(r, b=bufs, M=M, N=N, K=K, G=G):
@@ -885,6 +895,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config timings")
     ap.add_argument("--configs", default="", help="comma-separated subset of the per-config timings")
+    ap.add_argument("--cold-activations", action="store_true",
+                    help="rotate the activations with the weights (from HBM) instead of one L2-resident buffer")
     ap.add_argument("--no-tune", action="store_true",
                     help="per-config timings with the built-in heuristic instead of autotuned launch forms")
     ap.add_argument("--tune-headline", action="store_true",
