@@ -242,7 +242,8 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
                     }
                 }
             }
-            const int gr = (kr0 + i * kBlockK) / p.G - g_lo;
+            const int gr =
+                static_cast<int>((static_cast<uint64_t>(kr0 + i * kBlockK) * p.g_magic) >> 32) - g_lo;  // floor(k / G)
             const float sa = __half2float(scl[gr * 128 + ja]);
             const float sb = __half2float(scl[gr * 128 + ja + 8]);
 #pragma unroll
