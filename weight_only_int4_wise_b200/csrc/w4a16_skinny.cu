@@ -175,20 +175,46 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
         for (int i = 0; i < kDepth; ++i) issue_block(i);
     }
     {
+        // 16-byte chunks (row r, chunk c) of the CTA's K range, kThreads apart per
+        // thread, walked without a division per chunk; each batch's loads go out
+        // together, so a batch costs one memory round trip on this critical path.
         const int cpr = krange / 8;  // 16-byte chunks per activation row
-        for (int idx = threadIdx.x; idx < MP * cpr; idx += kThreads) {
-            const int r = idx / cpr, c = idx - r * cpr;
-            const int k = kr0 + c * 8;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (r < Mrows && k < p.K) v = *reinterpret_cast<const uint4*>(Ap + static_cast<int64_t>(r) * p.K + k);
-            // Within each 128-deep block the 4-wide k groups are interleaved: group
-            // (t, s) (k = 32t + 4s .. +3, thread column t's step s) sits at halves
-            // 16s + 4t. With rows 16 halves (32 bytes mod 128) apart, the 32 lanes'
-            // 8-byte fragment loads of one step then hit distinct banks.
-            const int q = c & 3, t4 = (c >> 2) & 3;
-            __half* rowp = act + r * p.act_stride + (c >> 4) * 128 + 32 * q + 4 * t4;
-            *reinterpret_cast<uint2*>(rowp) = make_uint2(v.x, v.y);
-            *reinterpret_cast<uint2*>(rowp + 16) = make_uint2(v.z, v.w);
+        const int total = MP * cpr;
+        int r = static_cast<int>(threadIdx.x) / cpr;
+        int c = static_cast<int>(threadIdx.x) - r * cpr;
+        const int rstep = kThreads / cpr, cstep = kThreads - rstep * cpr;
+        constexpr int kBatch = 4;
+        for (int idx0 = threadIdx.x; idx0 < total; idx0 += kBatch * kThreads) {
+            uint4 v[kBatch];
+            int rr[kBatch], cc[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                rr[u] = r;
+                cc[u] = c;
+                const int k = kr0 + c * 8;
+                v[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (idx0 + u * kThreads < total && r < Mrows && k < p.K)
+                    v[u] = *reinterpret_cast<const uint4*>(Ap + static_cast<int64_t>(r) * p.K + k);
+                c += cstep;
+                r += rstep;
+                if (c >= cpr) {
+                    c -= cpr;
+                    ++r;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                if (idx0 + u * kThreads < total) {
+                    // Within each 128-deep block the 4-wide k groups are interleaved: group
+                    // (t, s) (k = 32t + 4s .. +3, thread column t's step s) sits at halves
+                    // 16s + 4t. With rows 16 halves (32 bytes mod 128) apart, the 32 lanes'
+                    // 8-byte fragment loads of one step then hit distinct banks.
+                    const int q = cc[u] & 3, t4 = (cc[u] >> 2) & 3;
+                    __half* rowp = act + rr[u] * p.act_stride + (cc[u] >> 4) * 128 + 32 * q + 4 * t4;
+                    *reinterpret_cast<uint2*>(rowp) = make_uint2(v[u].x, v[u].y);
+                    *reinterpret_cast<uint2*>(rowp + 16) = make_uint2(v[u].z, v[u].w);
+                }
+            }
         }
     }
     cp_async_wait<kDepth - 1>();  // the scale rows (and this thread's first block) have landed
