@@ -24,8 +24,8 @@
 //
 // The quotient w / s decides an integer, so it must be the IEEE one: the
 // kernels take w * (1/s) (within 2 ulp of it) and fall back to the IEEE
-// division only when that product lies within 1e-5 of a rounding boundary
-// (a half-integer); elsewhere both round to the same integer.
+// division only when that product lies within 1e-5 (8-bit codes: 1e-4) of a
+// rounding boundary (a half-integer); elsewhere both round to the same integer.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -61,13 +61,17 @@ struct QuantRange {
 
 // Code of weight w with scale s (inverse rs = 1/s rounded): round(w / s), halves
 // away from zero, clamped to the code range; 0 when s = 0.
+// Away from a half-integer the quotient's nearest integer (rintf of w * (1/s))
+// is the rounded code under any tie rule: the true quotient is within 2 ulp of
+// the product, far inside the window. Near a half-integer the IEEE quotient
+// decides, with halves away from zero.
 template <int BITS>
 __device__ __forceinline__ uint32_t quantize_code(float w, float s, float rs) {
     if (s == 0.0f) return 0u;
-    float x = w * rs;
-    const float a = fabsf(x);
-    if (fabsf(a - floorf(a) - 0.5f) < QuantRange<BITS>::kWindow) x = __fdiv_rn(w, s);
-    int q = static_cast<int>(roundf(x));
+    const float x = w * rs;
+    float r = rintf(x);
+    if (fabsf(x - r) > 0.5f - QuantRange<BITS>::kWindow) r = roundf(__fdiv_rn(w, s));
+    int q = static_cast<int>(r);
     q = q < QuantRange<BITS>::kMin ? QuantRange<BITS>::kMin : (q > QuantRange<BITS>::kMax ? QuantRange<BITS>::kMax : q);
     return static_cast<uint32_t>(q) & (BITS == 4 ? 0xFu : 0xFFu);
 }
