@@ -36,6 +36,10 @@ def empty_table():
     (8, 2048, 1024, 48),     # groups that straddle the 128-deep blocks
     (40, 1024, 512, 64),     # the tensor-core kernel with K splits over one token tile
     (300, 512, 392, 128),    # several token tiles, ragged last column tile
+    (5, 1000, 4696, 48),     # 37 column tiles, groups finer than a block, ragged K and N
+    (13, 960, 4696, 64),     # two token tiles, an odd count of 64-deep K tiles
+    (1, 2048, 4696, 256),    # one group per two blocks (scaled once per block)
+    (8, 4096, 14336, 128),   # the MLP up projection at full size
 ])
 def test_every_tactic_matches_the_oracle(o, M, K, N, G):
     c = workloads.dense(M, K, N, G, seed=M + K + N)

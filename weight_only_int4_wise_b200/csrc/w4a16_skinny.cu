@@ -110,8 +110,8 @@ __global__ void __launch_bounds__(KH * kSkThreads, 2)
     const int kh = static_cast<int>(threadIdx.x) / kSkThreads;  // K half: blocks i with i % KH == kh
     const int g = lane >> 2, t = lane & 3;
     const int split = blockIdx.x, nt = blockIdx.y;
-    const int b0 = static_cast<int>((static_cast<int64_t>(split) * p.KB) / p.splits);
-    const int b1 = static_cast<int>((static_cast<int64_t>(split + 1) * p.KB) / p.splits);
+    const int b0 = (split * p.KB) / p.splits;  // (32-bit: K < 2^31, so KB < 2^24)
+    const int b1 = ((split + 1) * p.KB) / p.splits;
     const int nb = b1 - b0;
     const int kr0 = b0 * kBlockK;                   // first k of this CTA
     const int krange = nb * kBlockK;
