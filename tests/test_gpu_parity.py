@@ -261,6 +261,42 @@ def test_quantize_bit_exact(o, K, N, G):
     assert np.array_equal(wp.cpu().numpy(), ref_wp)
 
 
+def rounding_boundary_case(K, N, G, top):
+    """Weights on and next to every rounding boundary of the code range: in each
+    group of each column the maximum |w| is top * s with s a power of two, so the
+    fp16 scale is exactly s and w / s is exact. The other rows cycle through the
+    half-integers of the range (ties, rounded away from zero), their fp16
+    neighbours on both sides, and the integers."""
+    halves = np.arange(-top, top) + 0.5  # (|w| <= top * s, so the maximum stays top * s)
+    base = np.concatenate([halves, np.arange(-top, top + 1).astype(np.float64)])
+    W = np.zeros((K, N), dtype=np.float16)
+    for n in range(N):
+        s = 2.0 ** (-(n % 6) - 3)
+        vals = (base * s).astype(np.float16)
+        up = np.nextafter(vals[:len(halves)], np.float16(np.inf))
+        down = np.nextafter(vals[:len(halves)], np.float16(-np.inf))
+        cyc = np.concatenate([vals, up, down])
+        cyc = np.roll(cyc, n)
+        for g0 in range(0, K, G):
+            rows = min(G, K - g0)
+            col = np.resize(cyc, rows)
+            col[0] = np.float16((top if (g0 // G + n) % 2 == 0 else -top) * s)
+            W[g0:g0 + rows, n] = col
+    return W
+
+
+@pytest.mark.parametrize("K,N,G", [(512, 264, 64), (130, 24, 128)])
+def test_quantize_rounding_boundaries(o, K, N, G):
+    # every tie and its neighbours, on the staged (N % 8 == 0) and fallback forms
+    W = rounding_boundary_case(K, N, G, top=7)
+    wp, S = w.quantize(dev(W), G)
+    torch.cuda.synchronize()
+    ref_wp, ref_S = o.quantize(W, G)
+    assert np.all(ref_S.astype(np.float32) > 0)
+    assert np.array_equal(S.cpu().numpy().view(np.uint16), ref_S.view(np.uint16))
+    assert np.array_equal(wp.cpu().numpy(), ref_wp)
+
+
 def test_quantize_worked_example():
     # the hand-worked example (tests/golden/quantize_example.txt), one zero column added (N even)
     dims, t = pins._read_quantize_example()

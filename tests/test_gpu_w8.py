@@ -71,6 +71,19 @@ def test_w8_quantize_bit_exact(o, K, N, G):
     assert w.device_status() == w.OK
 
 
+@pytest.mark.parametrize("K,N,G", [(1024, 264, 256), (300, 40, 128)])
+def test_w8_quantize_rounding_boundaries(o, K, N, G):
+    # every tie of the 8-bit range and its fp16 neighbours, staged and fallback forms
+    from test_gpu_parity import rounding_boundary_case
+    W = rounding_boundary_case(K, N, G, top=127)
+    q8, S = w.quantize_w8(dev(W), G)
+    torch.cuda.synchronize()
+    ref_q, ref_S = o.quantize_w8(W, G)
+    assert np.array_equal(S.cpu().numpy().view(np.uint16), ref_S.view(np.uint16))
+    assert np.array_equal(q8.cpu().numpy(), ref_q)
+    assert w.device_status() == w.OK
+
+
 def test_w8_quantize_then_gemm(o):
     # the export chain: fp16 weights -> 8-bit codes and scales -> tiled layout -> product
     M, K, N, G = 24, 1024, 512, 128

@@ -61,17 +61,23 @@ struct QuantRange {
 
 // Code of weight w with scale s (inverse rs = 1/s rounded): round(w / s), halves
 // away from zero, clamped to the code range; 0 when s = 0.
-// Away from a half-integer the quotient's nearest integer (rintf of w * (1/s))
+// Away from a half-integer the quotient's nearest integer (that of w * (1/s))
 // is the rounded code under any tie rule: the true quotient is within 2 ulp of
 // the product, far inside the window. Near a half-integer the IEEE quotient
 // decides, with halves away from zero.
+// The nearest integer of x comes from the magic-number method: for |x| < 2^22
+// the float sum x + 1.5 * 2^23 lies in [2^23, 2^24), where the spacing is 1, so
+// the sum is rounded to an integer (ties to even) and its bit pattern is
+// 0x4B400000 + that integer; subtracting 1.5 * 2^23 again gives it as a float.
+// (|x| stays far below 2^22: at most about 2 * 127 for 8-bit codes.)
 template <int BITS>
 __device__ __forceinline__ uint32_t quantize_code(float w, float s, float rs) {
     if (s == 0.0f) return 0u;
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23, bit pattern 0x4B400000
     const float x = w * rs;
-    float r = rintf(x);
-    if (fabsf(x - r) > 0.5f - QuantRange<BITS>::kWindow) r = roundf(__fdiv_rn(w, s));
-    int q = static_cast<int>(r);
+    const float m = x + kMagic;
+    int q = __float_as_int(m) - 0x4B400000;
+    if (fabsf(x - (m - kMagic)) > 0.5f - QuantRange<BITS>::kWindow) q = static_cast<int>(roundf(__fdiv_rn(w, s)));
     q = q < QuantRange<BITS>::kMin ? QuantRange<BITS>::kMin : (q > QuantRange<BITS>::kMax ? QuantRange<BITS>::kMax : q);
     return static_cast<uint32_t>(q) & (BITS == 4 ? 0xFu : 0xFFu);
 }
@@ -95,22 +101,24 @@ __device__ __forceinline__ void quantize_pair(RowFn row, int64_t nrows, uint16_t
     const float2 s = __half22float2(sh);
     const float r0 = s.x != 0.0f ? __frcp_rn(s.x) : 0.0f;
     const float r1 = s.y != 0.0f ? __frcp_rn(s.y) : 0.0f;
+    // (nrows is at most G rows of one group, below 2^31)
+    const int n = static_cast<int>(nrows);
+    uint16_t* out = out_row0;
     if constexpr (BITS == 4) {
         // Row pairs (k, k + 1): groups start on even rows (G is even), so a packed
         // byte never spans two groups; a missing last odd row packs 0.
-        for (int64_t r = 0; r < nrows; r += 2) {
+        for (int r = 0; r < n; r += 2, out += N2) {
             const float2 lo = __half22float2(row(r));
-            const bool two = r + 1 < nrows;
+            const bool two = r + 1 < n;
             const float2 hi = two ? __half22float2(row(r + 1)) : make_float2(0.0f, 0.0f);
             const uint32_t b0 = quantize_code<4>(lo.x, s.x, r0) | (two ? quantize_code<4>(hi.x, s.x, r0) << 4 : 0u);
             const uint32_t b1 = quantize_code<4>(lo.y, s.y, r1) | (two ? quantize_code<4>(hi.y, s.y, r1) << 4 : 0u);
-            out_row0[(r >> 1) * N2] = static_cast<uint16_t>(b0 | (b1 << 8));  // bytes of the pair's two columns
+            *out = static_cast<uint16_t>(b0 | (b1 << 8));  // bytes of the pair's two columns
         }
     } else {
-        for (int64_t r = 0; r < nrows; ++r) {
+        for (int r = 0; r < n; ++r, out += N2) {
             const float2 v = __half22float2(row(r));
-            out_row0[r * N2] =
-                static_cast<uint16_t>(quantize_code<8>(v.x, s.x, r0) | (quantize_code<8>(v.y, s.y, r1) << 8));
+            *out = static_cast<uint16_t>(quantize_code<8>(v.x, s.x, r0) | (quantize_code<8>(v.y, s.y, r1) << 8));
         }
     }
 }
@@ -170,12 +178,11 @@ __global__ void __launch_bounds__(kQuantThreads * kSlices) quantize_tma_kernel(c
         const int64_t per = ((nrows + kSlices - 1) / kSlices + 1) & ~int64_t(1);
         const int64_t r0 = slice * per < nrows ? slice * per : nrows;
         const int64_t r1 = r0 + per < nrows ? r0 + per : nrows;
-        float a0 = 0.0f, a1 = 0.0f;
-        for (int64_t r = r0; r < r1; ++r) {
-            const float2 v = __half22float2(tile[r * kQuantThreads + t]);
-            a0 = fmaxf(a0, fabsf(v.x));
-            a1 = fmaxf(a1, fabsf(v.y));
-        }
+        // The slice's maxima of |w| in fp16 (exact: no rounding in abs or max).
+        __half2 amax = __float2half2_rn(0.0f);
+        for (int r = static_cast<int>(r0); r < static_cast<int>(r1); ++r)
+            amax = __hmax2(amax, __habs2(tile[r * kQuantThreads + t]));
+        float a0 = __low2float(amax), a1 = __high2float(amax);
         part[slice * kQuantThreads + t] = make_float2(a0, a1);
         __syncthreads();
 #pragma unroll
