@@ -417,8 +417,10 @@ def run_ours(args):
     # GEMM out of the programmatic-dependent-launch overlap with the kernel before
     # it; per-step copies cost about 4 us per step that way.) E2E_GRAPH_STEPS
     # steps, rotating weight copies as in the timed region, are recorded once
-    # into a CUDA graph and replayed.
-    E2E_BATCH, E2E_GRAPH_STEPS = 8, 32
+    # into a CUDA graph and replayed. Replays run one after another, so each
+    # one starts with a batch copy-in that nothing overlaps and ends with a
+    # copy-out: a long graph spreads those two over more steps.
+    E2E_BATCH, E2E_GRAPH_STEPS = 8, 128
     rows_step = 1 + 16
     A_step = np.concatenate([case.A[:1], case.A], axis=0)
     A_h = torch.from_numpy(np.concatenate([A_step] * E2E_BATCH, axis=0)).pin_memory()
