@@ -59,8 +59,10 @@ struct QuantRange {
     static constexpr float kWindow = BITS == 4 ? 1e-5f : 1e-4f;
 };
 
-// Code of weight w with scale s (inverse rs = 1/s rounded): round(w / s), halves
-// away from zero, clamped to the code range; 0 when s = 0.
+// Code of weight w with scale s (inverse rs = 1/s rounded, 0 when s = 0):
+// round(w / s), halves away from zero, clamped to the code range; 0 when s = 0
+// (then x = w * 0 = 0 for finite w, whose nearest integer is 0 with no
+// boundary to check).
 // Away from a half-integer the quotient's nearest integer (that of w * (1/s))
 // is the rounded code under any tie rule: the true quotient is within 2 ulp of
 // the product, far inside the window. Near a half-integer the IEEE quotient
@@ -72,7 +74,6 @@ struct QuantRange {
 // (|x| stays far below 2^22: at most about 2 * 127 for 8-bit codes.)
 template <int BITS>
 __device__ __forceinline__ uint32_t quantize_code(float w, float s, float rs) {
-    if (s == 0.0f) return 0u;
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23, bit pattern 0x4B400000
     const float x = w * rs;
     const float m = x + kMagic;
@@ -107,15 +108,21 @@ __device__ __forceinline__ void quantize_pair(RowFn row, int64_t nrows, uint16_t
     if constexpr (BITS == 4) {
         // Row pairs (k, k + 1): groups start on even rows (G is even), so a packed
         // byte never spans two groups; a missing last odd row packs 0.
-        for (int r = 0; r < n; r += 2, out += N2) {
+        const int full = n & ~1;
+#pragma unroll 4
+        for (int r = 0; r < full; r += 2, out += N2) {
             const float2 lo = __half22float2(row(r));
-            const bool two = r + 1 < n;
-            const float2 hi = two ? __half22float2(row(r + 1)) : make_float2(0.0f, 0.0f);
-            const uint32_t b0 = quantize_code<4>(lo.x, s.x, r0) | (two ? quantize_code<4>(hi.x, s.x, r0) << 4 : 0u);
-            const uint32_t b1 = quantize_code<4>(lo.y, s.y, r1) | (two ? quantize_code<4>(hi.y, s.y, r1) << 4 : 0u);
+            const float2 hi = __half22float2(row(r + 1));
+            const uint32_t b0 = quantize_code<4>(lo.x, s.x, r0) | (quantize_code<4>(hi.x, s.x, r0) << 4);
+            const uint32_t b1 = quantize_code<4>(lo.y, s.y, r1) | (quantize_code<4>(hi.y, s.y, r1) << 4);
             *out = static_cast<uint16_t>(b0 | (b1 << 8));  // bytes of the pair's two columns
         }
+        if (n & 1) {
+            const float2 lo = __half22float2(row(full));
+            *out = static_cast<uint16_t>(quantize_code<4>(lo.x, s.x, r0) | (quantize_code<4>(lo.y, s.y, r1) << 8));
+        }
     } else {
+#pragma unroll 4
         for (int r = 0; r < n; ++r, out += N2) {
             const float2 v = __half22float2(row(r));
             *out = static_cast<uint16_t>(quantize_code<8>(v.x, s.x, r0) | (quantize_code<8>(v.y, s.y, r1) << 8));
