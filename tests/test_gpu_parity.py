@@ -297,6 +297,28 @@ def test_quantize_rounding_boundaries(o, K, N, G):
     assert np.array_equal(wp.cpu().numpy(), ref_wp)
 
 
+def subnormal_scale_case(K, N, G, lo, hi, seed):
+    """Weights that are small multiples of 2^-24 (fp16 subnormals): the group
+    scales are subnormal too, their rounding is coarse, and quotients beyond the
+    code range occur, so the clamp decides codes."""
+    g = np.random.Generator(np.random.PCG64(seed))
+    units = g.integers(lo, hi + 1, size=(1, N))
+    k = np.rint(g.uniform(-1.0, 1.0, size=(K, N)) * units)
+    return (k * 2.0 ** -24).astype(np.float16)
+
+
+@pytest.mark.parametrize("K,N,G", [(256, 264, 64), (130, 24, 128)])
+def test_quantize_subnormal_scales(o, K, N, G):
+    W = subnormal_scale_case(K, N, G, lo=3, hi=40, seed=K + N)
+    wp, S = w.quantize(dev(W), G)
+    torch.cuda.synchronize()
+    ref_wp, ref_S = o.quantize(W, G)
+    q = o.unpack(ref_wp, K)
+    assert np.any(q == 7) and np.any(q == -8)  # the clamp is reached
+    assert np.array_equal(S.cpu().numpy().view(np.uint16), ref_S.view(np.uint16))
+    assert np.array_equal(wp.cpu().numpy(), ref_wp)
+
+
 def test_quantize_worked_example():
     # the hand-worked example (tests/golden/quantize_example.txt), one zero column added (N even)
     dims, t = pins._read_quantize_example()

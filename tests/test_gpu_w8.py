@@ -84,6 +84,20 @@ def test_w8_quantize_rounding_boundaries(o, K, N, G):
     assert w.device_status() == w.OK
 
 
+@pytest.mark.parametrize("K,N,G", [(256, 264, 64), (300, 40, 128)])
+def test_w8_quantize_subnormal_scales(o, K, N, G):
+    # subnormal scales, coarsely rounded: the clamp to [-128, 127] decides codes
+    from test_gpu_parity import subnormal_scale_case
+    W = subnormal_scale_case(K, N, G, lo=100, hi=260, seed=K * 3 + N)
+    q8, S = w.quantize_w8(dev(W), G)
+    torch.cuda.synchronize()
+    ref_q, ref_S = o.quantize_w8(W, G)
+    assert np.any(ref_q == 127) and np.any(ref_q == -128)
+    assert np.array_equal(S.cpu().numpy().view(np.uint16), ref_S.view(np.uint16))
+    assert np.array_equal(q8.cpu().numpy(), ref_q)
+    assert w.device_status() == w.OK
+
+
 def test_w8_quantize_then_gemm(o):
     # the export chain: fp16 weights -> 8-bit codes and scales -> tiled layout -> product
     M, K, N, G = 24, 1024, 512, 128

@@ -72,15 +72,31 @@ struct QuantRange {
 // the sum is rounded to an integer (ties to even) and its bit pattern is
 // 0x4B400000 + that integer; subtracting 1.5 * 2^23 again gives it as a float.
 // (|x| stays far below 2^22: at most about 2 * 127 for 8-bit codes.)
-template <int BITS>
+// Returns a word whose low BITS bits are the code (two's complement).
+// CLAMP = false leaves out the clamp, for groups whose scale is 0 or a normal
+// fp16 number: then s >= (max / kMax) (1 - 2^-11) (one fp16 and one float
+// rounding), so |w| <= max gives |w * (1/s)| <= kMax (1 + 2^-10) < kMax + 0.5,
+// and the rounded code is already in range. Below 2^-14 (subnormal scales) the
+// fp16 rounding error is relatively larger and the clamp is needed. Without
+// the clamp the code is read straight from the low bits of the magic sum
+// (0x4B400000 is a multiple of 256, so those bits are the integer's own).
+template <int BITS, bool CLAMP>
 __device__ __forceinline__ uint32_t quantize_code(float w, float s, float rs) {
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23, bit pattern 0x4B400000
     const float x = w * rs;
     const float m = x + kMagic;
-    int q = __float_as_int(m) - 0x4B400000;
-    if (fabsf(x - (m - kMagic)) > 0.5f - QuantRange<BITS>::kWindow) q = static_cast<int>(roundf(__fdiv_rn(w, s)));
-    q = q < QuantRange<BITS>::kMin ? QuantRange<BITS>::kMin : (q > QuantRange<BITS>::kMax ? QuantRange<BITS>::kMax : q);
-    return static_cast<uint32_t>(q) & (BITS == 4 ? 0xFu : 0xFFu);
+    int q = __float_as_int(m);
+    const bool boundary = fabsf(x - (m - kMagic)) > 0.5f - QuantRange<BITS>::kWindow;
+    if constexpr (CLAMP) {
+        q -= 0x4B400000;
+        if (boundary) q = static_cast<int>(roundf(__fdiv_rn(w, s)));
+        q = q < QuantRange<BITS>::kMin ? QuantRange<BITS>::kMin
+                                       : (q > QuantRange<BITS>::kMax ? QuantRange<BITS>::kMax : q);
+        return static_cast<uint32_t>(q) & (BITS == 4 ? 0xFu : 0xFFu);
+    } else {
+        if (boundary) q = static_cast<int>(roundf(__fdiv_rn(w, s)));
+        return static_cast<uint32_t>(q);
+    }
 }
 
 template <int BITS>
@@ -94,6 +110,40 @@ __device__ __forceinline__ __half2 group_scales(float a0, float a1) {
 // from out_row0 on with a stride of N2 16-bit words per output row: for int4 one
 // packed byte per column and row pair (rows of the canonical packed layout), for
 // 8-bit codes one byte per column and row.
+// The codes of rows 0..n-1 of one column pair with scales s and inverses
+// (r0, r1), written from out on with a stride of N2 16-bit words per row.
+template <int BITS, bool CLAMP, typename RowFn>
+__device__ __forceinline__ void quantize_rows(RowFn row, int n, uint16_t* __restrict__ out, int64_t N2, float2 s,
+                                              float r0, float r1) {
+    if constexpr (BITS == 4) {
+        // Row pairs (k, k + 1): groups start on even rows (G is even), so a packed
+        // byte never spans two groups; a missing last odd row packs 0.
+        const int full = n & ~1;
+#pragma unroll 4
+        for (int r = 0; r < full; r += 2, out += N2) {
+            const float2 lo = __half22float2(row(r));
+            const float2 hi = __half22float2(row(r + 1));
+            const uint32_t b0 = (quantize_code<4, CLAMP>(lo.x, s.x, r0) & 0xFu) |
+                                ((quantize_code<4, CLAMP>(hi.x, s.x, r0) & 0xFu) << 4);
+            const uint32_t b1 = (quantize_code<4, CLAMP>(lo.y, s.y, r1) & 0xFu) |
+                                ((quantize_code<4, CLAMP>(hi.y, s.y, r1) & 0xFu) << 4);
+            *out = static_cast<uint16_t>(b0 | (b1 << 8));  // bytes of the pair's two columns
+        }
+        if (n & 1) {
+            const float2 lo = __half22float2(row(full));
+            *out = static_cast<uint16_t>((quantize_code<4, CLAMP>(lo.x, s.x, r0) & 0xFu) |
+                                         ((quantize_code<4, CLAMP>(lo.y, s.y, r1) & 0xFu) << 8));
+        }
+    } else {
+#pragma unroll 4
+        for (int r = 0; r < n; ++r, out += N2) {
+            const float2 v = __half22float2(row(r));
+            *out = static_cast<uint16_t>((quantize_code<8, CLAMP>(v.x, s.x, r0) & 0xFFu) |
+                                         ((quantize_code<8, CLAMP>(v.y, s.y, r1) & 0xFFu) << 8));
+        }
+    }
+}
+
 template <int BITS, typename RowFn>
 __device__ __forceinline__ void quantize_pair(RowFn row, int64_t nrows, uint16_t* __restrict__ out_row0,
                                               int64_t N2, __half2* __restrict__ s_out, float a0, float a1) {
@@ -104,30 +154,12 @@ __device__ __forceinline__ void quantize_pair(RowFn row, int64_t nrows, uint16_t
     const float r1 = s.y != 0.0f ? __frcp_rn(s.y) : 0.0f;
     // (nrows is at most G rows of one group, below 2^31)
     const int n = static_cast<int>(nrows);
-    uint16_t* out = out_row0;
-    if constexpr (BITS == 4) {
-        // Row pairs (k, k + 1): groups start on even rows (G is even), so a packed
-        // byte never spans two groups; a missing last odd row packs 0.
-        const int full = n & ~1;
-#pragma unroll 4
-        for (int r = 0; r < full; r += 2, out += N2) {
-            const float2 lo = __half22float2(row(r));
-            const float2 hi = __half22float2(row(r + 1));
-            const uint32_t b0 = quantize_code<4>(lo.x, s.x, r0) | (quantize_code<4>(hi.x, s.x, r0) << 4);
-            const uint32_t b1 = quantize_code<4>(lo.y, s.y, r1) | (quantize_code<4>(hi.y, s.y, r1) << 4);
-            *out = static_cast<uint16_t>(b0 | (b1 << 8));  // bytes of the pair's two columns
-        }
-        if (n & 1) {
-            const float2 lo = __half22float2(row(full));
-            *out = static_cast<uint16_t>(quantize_code<4>(lo.x, s.x, r0) | (quantize_code<4>(lo.y, s.y, r1) << 8));
-        }
-    } else {
-#pragma unroll 4
-        for (int r = 0; r < n; ++r, out += N2) {
-            const float2 v = __half22float2(row(r));
-            *out = static_cast<uint16_t>(quantize_code<8>(v.x, s.x, r0) | (quantize_code<8>(v.y, s.y, r1) << 8));
-        }
-    }
+    constexpr float kMinNormal = 6.103515625e-05f;  // 2^-14, the smallest normal fp16 number
+    const bool in_range = (s.x == 0.0f || s.x >= kMinNormal) && (s.y == 0.0f || s.y >= kMinNormal);
+    if (in_range)
+        quantize_rows<BITS, false>(row, n, out_row0, N2, s, r0, r1);
+    else
+        quantize_rows<BITS, true>(row, n, out_row0, N2, s, r0, r1);
 }
 
 // Group g of a 256-column tile through shared memory (see the file header).
